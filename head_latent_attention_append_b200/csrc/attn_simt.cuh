@@ -1,0 +1,201 @@
+// Absorbed latent attention on CUDA cores (fp32 FFMA), split-KV.
+//
+// This is the fp32 path (the fp32 workload's 1e-4 bound rules out single-pass
+// TF32 on the tensor cores).  Per query token and head it computes
+//   a_t   = Q_abs[h] . cache[t]          over the d_c + d_r columns
+//           (Q_abs = [s*log2(e)*W_UK,h^T q_C,h | s*log2(e)*RoPE_m(q_R,h)], so
+//           a_t is the pages' score in log2 units)
+//   alpha = softmax over the visible keys (exp2, online, running max)
+//   obar  = sum_t alpha_t c_t            over the d_c latent columns
+// ("ai-decoupled-rope-mla": absorbed score and output equations).
+//
+// Grid: (worker, head group).  A CTA walks its worker's segments (sched.cuh)
+// for HG heads; 32 keys at a time are staged in shared memory as fp32.
+#pragma once
+#include "common.cuh"
+#include "sched.cuh"
+
+namespace mla {
+
+struct AttnArgs {
+  const void* qabs;          // [R][qrows][d_cr]
+  int qrows;
+  const void* cache;         // [num_pages][page_size][d_cr]
+  const int32_t* page_table; // [n_seq][max_pages]
+  int max_pages, num_pages, page_size;
+  int n_h, d_c, d_r, d_cr;
+  const int32_t* kv_len;
+  int uniform_kv_len, n_q, max_kv_len;
+  Sched sched;
+  float* part_o;             // [2W][n_h][d_c]
+  float* part_ml;            // [2W][n_h][2]
+  void* obar;                // [R][n_h][d_c] (type of the path)
+  int* err;
+};
+
+namespace attn_simt {
+constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(THREADS) kernel(AttnArgs a, int HG) {
+  extern __shared__ float smem[];
+  const int pitch = a.d_cr + 1;
+  float* Qs = smem;                    // [HG][pitch]
+  float* Cs = Qs + HG * pitch;         // [KC][pitch]
+  float* Ps = Cs + KC * pitch;         // [HG][KC]
+  float* st = Ps + HG * KC;            // [HG][3]: m, l, corr
+  const int w = blockIdx.x, h0 = blockIdx.y * HG;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int TPH = THREADS / HG;        // threads per head in the output update
+  const int oh = tid / TPH, oj = tid % TPH;
+  const int cpt = ceil_div(a.d_c, TPH);  // <= MAX_CPT (d_c <= 512, TPH >= 16)
+  const T* qabs = static_cast<const T*>(a.qabs);
+  const T* cache = static_cast<const T*>(a.cache);
+  const Sched& S = a.sched;
+
+  for (int si = S.worker_seg[w]; si < S.worker_seg[w + 1]; ++si) {
+    const Seg g = S.segs[si];
+    const int rb = g.rb, seq = rb / a.n_q;
+    const int nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
+    __syncthreads();
+    for (int i = tid; i < HG * a.d_cr; i += THREADS) {
+      int h = i / a.d_cr, j = i % a.d_cr;
+      Qs[h * pitch + j] = (h0 + h < a.n_h) ? to_f32(qabs[((long long)rb * a.qrows + h0 + h) * a.d_cr + j]) : 0.f;
+    }
+    if (tid < HG) {
+      st[tid * 3 + 0] = -INFINITY;
+      st[tid * 3 + 1] = 0.f;
+    }
+    float o[MAX_CPT];
+#pragma unroll
+    for (int r = 0; r < MAX_CPT; ++r) o[r] = 0.f;
+
+    const int k_begin = g.t_lo * a.page_size;
+    const int k_end = min(nkeys, g.t_hi * a.page_size);
+    for (int k0 = k_begin; k0 < k_end; k0 += KC) {
+      __syncthreads();
+      // Stage KC cache rows (positions k0 .. k0+KC-1) through the page table.
+      for (int i = tid; i < KC * a.d_cr; i += THREADS) {
+        int k = i / a.d_cr, j = i % a.d_cr, p = k0 + k;
+        float v = 0.f;
+        if (p < k_end) {
+          int page = a.page_table[(long long)seq * a.max_pages + p / a.page_size];
+          if (page >= 0 && page < a.num_pages)
+            v = to_f32(cache[((long long)page * a.page_size + p % a.page_size) * a.d_cr + j]);
+          else if (j == 0)
+            flag_error(a.err, kErrBounds);
+        }
+        Cs[k * pitch + j] = v;
+      }
+      __syncthreads();
+      // Scores for HG x KC (head, key) pairs.
+      for (int i = tid; i < HG * KC; i += THREADS) {
+        int h = i / KC, k = i % KC;
+        const float* q = Qs + h * pitch;
+        const float* c = Cs + k * pitch;
+        float acc = 0.f;
+        for (int j = 0; j < a.d_cr; ++j) acc = fmaf(q[j], c[j], acc);
+        Ps[h * KC + k] = (k0 + k < k_end) ? acc : -INFINITY;
+      }
+      __syncthreads();
+      // Online softmax: one warp per head, one lane per key.
+      for (int h = warp; h < HG; h += THREADS / 32) {
+        float s = Ps[h * KC + lane];
+        float mx = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        float m_old = st[h * 3 + 0];
+        float m_new = fmaxf(m_old, mx);
+        float p = exp2f(s - m_new);
+        float sum = p;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        Ps[h * KC + lane] = p;
+        __syncwarp();
+        if (lane == 0) {
+          float corr = exp2f(m_old - m_new);
+          st[h * 3 + 0] = m_new;
+          st[h * 3 + 1] = st[h * 3 + 1] * corr + sum;
+          st[h * 3 + 2] = corr;
+        }
+      }
+      __syncthreads();
+      // obar[h][j] = obar*corr + sum_k P[h][k] * c[k][j].
+      if (oh < HG) {
+        const float corr = st[oh * 3 + 2];
+        const float* P = Ps + oh * KC;
+#pragma unroll
+        for (int r = 0; r < MAX_CPT; ++r) {
+          if (r < cpt && oj + r * TPH < a.d_c) {
+            int j = oj + r * TPH;
+            float acc = o[r] * corr;
+#pragma unroll 8
+            for (int k = 0; k < KC; ++k) acc = fmaf(P[k], Cs[k * pitch + j], acc);
+            o[r] = acc;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // Finish: a whole row block is normalised straight into obar; a piece of
+    // a split row block leaves (m, l, unnormalised sum) in its partial slot.
+    if (oh < HG && h0 + oh < a.n_h) {
+      const int h = h0 + oh;
+      const float m = st[oh * 3 + 0], l = st[oh * 3 + 1];
+      if (g.slot < 0) {
+        T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int r = 0; r < MAX_CPT; ++r)
+          if (r < cpt && oj + r * TPH < a.d_c) out[oj + r * TPH] = from_f32<T>(o[r] * inv);
+      } else {
+        float* po = a.part_o + ((long long)g.slot * a.n_h + h) * a.d_c;
+#pragma unroll
+        for (int r = 0; r < MAX_CPT; ++r)
+          if (r < cpt && oj + r * TPH < a.d_c) po[oj + r * TPH] = o[r];
+        if (oj == 0) {
+          a.part_ml[((long long)g.slot * a.n_h + h) * 2 + 0] = m;
+          a.part_ml[((long long)g.slot * a.n_h + h) * 2 + 1] = l;
+        }
+      }
+    }
+  }
+}
+
+inline size_t smem_bytes(int HG, int d_cr) {
+  return sizeof(float) * ((size_t)(HG + KC) * (d_cr + 1) + HG * KC + HG * 3);
+}
+}  // namespace attn_simt
+
+// ------------------------------------------------------------ combine -----
+// Merges the partial slots of each split row block (log-sum-exp in base 2):
+//   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  obar = sum_s 2^(m_s - m) O_s / l.
+// Slots are visited in segment order, so the result is deterministic.
+template <typename T>
+__global__ void combine_kernel(AttnArgs a) {
+  const Sched& S = a.sched;
+  const int idx = blockIdx.x;
+  if (idx >= S.split_rbs[0]) return;
+  const int rb = S.split_rbs[1 + idx], h = blockIdx.y;
+  const int s0 = S.rb_seg_first[rb], s1 = S.rb_seg_first[rb + 1];
+  float m = -INFINITY;
+  for (int s = s0; s < s1; ++s) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
+  float l = 0.f;
+  for (int s = s0; s < s1; ++s) {
+    const float* ml = a.part_ml + ((long long)S.segs[s].slot * a.n_h + h) * 2;
+    l += exp2f(ml[0] - m) * ml[1];
+  }
+  const float inv = 1.f / l;
+  T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
+  for (int j = threadIdx.x; j < a.d_c; j += blockDim.x) {
+    float acc = 0.f;
+    for (int s = s0; s < s1; ++s) {
+      int slot = S.segs[s].slot;
+      float wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
+      acc += wgt * a.part_o[((long long)slot * a.n_h + h) * a.d_c + j];
+    }
+    out[j] = from_f32<T>(acc * inv);
+  }
+}
+
+}  // namespace mla

@@ -1,0 +1,51 @@
+// Shared device helpers for libmla kernels (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace mla {
+
+// Bits OR-ed into the workspace error word by device-side checks.
+enum DeviceErr : int { kErrBounds = 1, kErrTimeout = 2 };
+
+__device__ __forceinline__ void flag_error(int* err_word, int bit) {
+  if (err_word) atomicOr(err_word, bit);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Stores two adjacent elements (index n even, 8- or 4-byte aligned pair).
+__device__ __forceinline__ void store_pair(float* p, float a, float b) {
+  *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+__device__ __forceinline__ void store_pair(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+
+// RoPE on one interleaved pair (x0, x1) = components (2i, 2i+1), rotated by
+// angle pos * theta_i.  The angle is formed and reduced to [-pi, pi] in fp64
+// (positions reach 2^15, where an fp32 angle would be off by ~4e-3 rad); the
+// sine and cosine of the reduced angle are taken in fp32.
+__device__ __forceinline__ void rope_rotate_pair(float& x0, float& x1, int pos, double theta) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double ang = (double)pos * theta;
+  double r = ang - two_pi * rint(ang / two_pi);
+  float s, c;
+  sincosf((float)r, &s, &c);
+  float y0 = x0 * c - x1 * s;
+  float y1 = x0 * s + x1 * c;
+  x0 = y0;
+  x1 = y1;
+}
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace mla

@@ -1,0 +1,516 @@
+// libmla C ABI: argument checks, workspace layout and launch sequencing.
+// Every step of the path runs in this library's kernels; the host code only
+// validates, carves the caller's workspace and launches on the caller's
+// stream.
+#include "../../include/mla.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "attn_simt.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "prep.cuh"
+#include "sched.cuh"
+
+using namespace mla;
+
+struct mla_weights {
+  mla_dims d;
+  float scale;         // softmax scale actually used
+  size_t esz;          // element size of the path (4 or 2)
+  void* dkr;           // [d_c + d_r][d_model]
+  void* dq;            // [d_cq][d_model] or null
+  void* uqr;           // [n_h*(d_h + d_r)][d_in]
+  void* ukt;           // [n_h][d_c][d_h]
+  void* uv;            // [n_h*d_v][d_c]
+  double theta[32];    // RoPE frequencies, theta_i = base^(-2i/d_r)
+};
+
+namespace {
+
+thread_local int g_launches = 0;
+
+// Event pairs bracketing the attention kernel while profiling is on.
+struct Profiler {
+  bool on = false;
+  int cap = 0, used = 0;
+  cudaEvent_t* ev = nullptr;  // 2 * cap
+};
+thread_local Profiler g_prof;
+
+void prof_mark(cudaStream_t st, bool start) {
+  if (!g_prof.on || g_prof.used >= g_prof.cap) return;
+  cudaEventRecord(g_prof.ev[2 * g_prof.used + (start ? 0 : 1)], st);
+  if (!start) ++g_prof.used;
+}
+
+constexpr int kWorkerSlots = 296;        // partial-slot capacity: 2 * kWorkerSlots
+constexpr int kSplitKTileSplits = 1024;  // split-K scratch: tiles * splits <= this
+constexpr int kCounterCap = 1024;
+constexpr double kLog2e = 1.4426950408889634074;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+mla_status check_dims(const mla_dims* d) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->n_h <= 0 || d->d_h <= 0 || d->d_v <= 0 || d->d_c <= 0 || d->d_r <= 0 || d->d_model <= 0 ||
+      d->d_cq < 0 || d->page_size <= 0 || !(d->rope_base > 0.f) || d->softmax_scale < 0.f)
+    return MLA_ERR_INVALID_ARG;
+  if (d->dtype != MLA_F32 && d->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
+  if (d->d_r % 2 != 0 || d->d_r > 64) return MLA_ERR_UNSUPPORTED;
+  if (d->page_size != 64) return MLA_ERR_UNSUPPORTED;
+  if (d->n_h > 128) return MLA_ERR_UNSUPPORTED;
+  if (d->dtype == MLA_BF16) {
+    // 16-byte row alignment for the tensor-core loads; d_c split evenly.
+    if (d->d_h % 8 || d->d_v % 8 || d->d_c % 64 || d->d_r % 16 || d->d_model % 8 || d->d_cq % 8)
+      return MLA_ERR_UNSUPPORTED;
+    if (d->d_c > 512) return MLA_ERR_UNSUPPORTED;
+  } else {
+    if (d->d_c > 512) return MLA_ERR_UNSUPPORTED;
+  }
+  return MLA_OK;
+}
+
+size_t esize(const mla_dims& d) { return d.dtype == MLA_BF16 ? 2 : 4; }
+int d_in(const mla_dims& d) { return d.d_cq > 0 ? d.d_cq : d.d_model; }
+
+struct WeightLayout {
+  size_t dkr, dq, uqr, ukt, uv, total;
+};
+WeightLayout weight_layout(const mla_dims& d) {
+  const size_t e = esize(d);
+  WeightLayout L{};
+  size_t o = 0;
+  L.dkr = o; o = align_up(o + e * (d.d_c + d.d_r) * d.d_model, 256);
+  L.dq = o;  o = align_up(o + e * (size_t)d.d_cq * d.d_model, 256);
+  L.uqr = o; o = align_up(o + e * (size_t)d.n_h * (d.d_h + d.d_r) * d_in(d), 256);
+  L.ukt = o; o = align_up(o + e * (size_t)d.n_h * d.d_c * d.d_h, 256);
+  L.uv = o;  o = align_up(o + e * (size_t)d.n_h * d.d_v * d.d_c, 256);
+  L.total = o;
+  return L;
+}
+
+// Workspace layout shared by the size queries and the calls.
+struct Plan {
+  size_t hdr, counters, partial, cq, qc, qabs, tile_start, worker_seg, segs, rb_first, split_rbs,
+      part_o, part_ml, obar, total;
+  int R, qrows;
+};
+Plan make_plan(const mla_dims& d, int R, bool attention) {
+  const size_t e = esize(d);
+  Plan P{};
+  P.R = R;
+  P.qrows = (d.dtype == MLA_BF16) ? 128 : d.n_h;
+  const int W = kWorkerSlots;
+  size_t o = 0;
+  P.hdr = o;        o = align_up(o + 256, 256);
+  P.counters = o;   o = align_up(o + sizeof(int) * kCounterCap, 256);
+  P.partial = o;    o = align_up(o + sizeof(float) * (size_t)kSplitKTileSplits * 64 * 64, 256);
+  if (attention) {
+    P.cq = o;         o = align_up(o + e * (size_t)R * d.d_cq, 256);
+    P.qc = o;         o = align_up(o + e * (size_t)R * d.n_h * d.d_h, 256);
+    P.qabs = o;       o = align_up(o + e * (size_t)R * P.qrows * (d.d_c + d.d_r), 256);
+    P.tile_start = o; o = align_up(o + sizeof(int) * (size_t)(R + 1), 256);
+    P.worker_seg = o; o = align_up(o + sizeof(int) * (size_t)(W + 1), 256);
+    P.segs = o;       o = align_up(o + sizeof(Seg) * (size_t)(W + R), 256);
+    P.rb_first = o;   o = align_up(o + sizeof(int) * (size_t)(R + 1), 256);
+    P.split_rbs = o;  o = align_up(o + sizeof(int) * (size_t)(2 * W + 1), 256);
+    P.part_o = o;     o = align_up(o + sizeof(float) * (size_t)2 * W * d.n_h * d.d_c, 256);
+    P.part_ml = o;    o = align_up(o + sizeof(float) * (size_t)2 * W * d.n_h * 2, 256);
+    P.obar = o;       o = align_up(o + e * (size_t)R * d.n_h * d.d_c, 256);
+  }
+  P.total = o;
+  return P;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// ----------------------------------------------------------- GEMM launcher
+template <typename T, class Epi>
+cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
+                 int M, int N, int K, int batch, const Epi& epi, void* ws, const Plan& P,
+                 cudaStream_t st) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  GemmArgs a{};
+  a.A = A; a.lda = lda; a.strideA = sA;
+  a.B = B; a.ldb = ldb; a.strideB = sB;
+  a.M = M; a.N = N; a.K = K; a.batch = batch;
+  const int tm = ceil_div(M, 64), tn = ceil_div(N, 64), tiles = tm * tn * batch;
+  int splits = 1;
+  const int want = 2 * num_sms();
+  if (tiles < want && tiles <= kCounterCap) {
+    splits = ceil_div(want, tiles);
+    splits = std::min(splits, std::max(1, K / 256));
+    splits = std::min(splits, kSplitKTileSplits / tiles);
+    splits = std::max(splits, 1);
+  }
+  int kchunk = ceil_div(ceil_div(K, splits), 32) * 32;
+  splits = ceil_div(K, kchunk);
+  a.splits = splits;
+  a.kchunk = kchunk;
+  a.partial = at<float>(ws, P.partial);
+  a.counters = at<int>(ws, P.counters);
+  dim3 grid(tn, tm, batch * splits);
+  ++g_launches;
+  if constexpr (sizeof(T) == 2) gemm_bf16::kernel<Epi><<<grid, gemm_bf16::THREADS, 0, st>>>(a, epi);
+  else gemm_f32::kernel<Epi><<<grid, gemm_f32::THREADS, 0, st>>>(a, epi);
+  return cudaGetLastError();
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------- pipelines
+template <typename T>
+mla_status append_impl(const mla_weights* w, const void* h, const int32_t* seq_idx, const int32_t* pos,
+                       int prefill_S, int n_seq, const int32_t* page_table, int max_pages, int num_pages,
+                       void* cache, int T_, void* ws, const Plan& P, cudaStream_t st) {
+  const mla_dims& d = w->d;
+  EpiAppend<T> epi{};
+  epi.cache = static_cast<T*>(cache);
+  epi.seq_idx = seq_idx;
+  epi.pos = pos;
+  epi.prefill_S = prefill_S;
+  epi.page_table = page_table;
+  for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
+  epi.max_pages = max_pages;
+  epi.num_pages = num_pages;
+  epi.page_size = d.page_size;
+  epi.d_c = d.d_c;
+  epi.d_cr = d.d_c + d.d_r;
+  epi.n_seq = n_seq;
+  epi.err = at<int>(ws, P.hdr);
+  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, d.d_c + d.d_r, d.d_model, 1, epi,
+                             ws, P, st));
+}
+
+template <typename T>
+mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_len, int uniform_kv_len,
+                       int n_q, int prefill_S, const int32_t* page_table, int max_pages, int num_pages,
+                       const void* cache, float* out, int R, int max_kv_len, void* ws, const Plan& P,
+                       cudaStream_t st) {
+  const mla_dims& d = w->d;
+  const int d_cr = d.d_c + d.d_r;
+  const int din = d_in(d);
+  int* err = at<int>(ws, P.hdr);
+  cudaError_t e;
+  // (1) query latent.
+  const void* src = hq;
+  if (d.d_cq > 0) {
+    EpiStore<T> epi{at<T>(ws, P.cq), d.d_cq, 0, 1.f};
+    if ((e = gemm<T>(hq, d.d_model, 0, w->dq, d.d_model, 0, R, d.d_cq, d.d_model, 1, epi, ws, P, st)))
+      return cuda_status(e);
+    src = at<T>(ws, P.cq);
+  }
+  // (2) q_C and rotated, scaled q_R.
+  const float qscale = (float)((double)w->scale * kLog2e);
+  {
+    EpiQProj<T> epi{};
+    epi.qc = at<T>(ws, P.qc);
+    epi.qabs = at<T>(ws, P.qabs);
+    epi.kv_len = kv_len;
+    epi.uniform_kv_len = uniform_kv_len;
+    for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
+    epi.n_h = d.n_h; epi.d_h = d.d_h; epi.d_r = d.d_r; epi.d_c = d.d_c; epi.d_cr = d_cr;
+    epi.qabs_rows = P.qrows; epi.n_q = n_q; epi.prefill_S = prefill_S;
+    epi.qr_scale = qscale;
+    if ((e = gemm<T>(src, din, 0, w->uqr, din, 0, R, d.n_h * (d.d_h + d.d_r), din, 1, epi, ws, P, st)))
+      return cuda_status(e);
+  }
+  // (3) absorption q~_h = W_UK,h^T q_C,h, scaled.
+  {
+    EpiStore<T> epi{at<T>(ws, P.qabs), (long long)P.qrows * d_cr, d_cr, qscale};
+    if ((e = gemm<T>(at<T>(ws, P.qc), (long long)d.n_h * d.d_h, d.d_h, w->ukt, d.d_h, (long long)d.d_c * d.d_h,
+                     R, d.d_c, d.d_h, d.n_h, epi, ws, P, st)))
+      return cuda_status(e);
+  }
+  // (4) schedule.
+  Sched S{at<int>(ws, P.tile_start), at<int>(ws, P.worker_seg), at<Seg>(ws, P.segs), at<int>(ws, P.rb_first),
+          at<int>(ws, P.split_rbs)};
+  AttnArgs aa{};
+  aa.qabs = at<T>(ws, P.qabs);
+  aa.qrows = P.qrows;
+  aa.cache = cache;
+  aa.page_table = page_table;
+  aa.max_pages = max_pages;
+  aa.num_pages = num_pages;
+  aa.page_size = d.page_size;
+  aa.n_h = d.n_h; aa.d_c = d.d_c; aa.d_r = d.d_r; aa.d_cr = d_cr;
+  aa.kv_len = kv_len; aa.uniform_kv_len = uniform_kv_len; aa.n_q = n_q; aa.max_kv_len = max_kv_len;
+  aa.sched = S;
+  aa.part_o = at<float>(ws, P.part_o);
+  aa.part_ml = at<float>(ws, P.part_ml);
+  aa.obar = at<T>(ws, P.obar);
+  aa.err = err;
+
+  // Heads per CTA: a power of two so that 256 threads split evenly.
+  int HG = 16;
+  while (HG > d.n_h) HG >>= 1;
+  const int G = ceil_div(d.n_h, HG);
+  int W = std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
+  {
+    SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
+    ++g_launches;
+    sched_kernel<<<1, 1024, 0, st>>>(sa);
+    if ((e = cudaGetLastError())) return cuda_status(e);
+  }
+  // (5) attention on the latent cache, (6) combine of split row blocks.
+  {
+    size_t sm = attn_simt::smem_bytes(HG, d_cr);
+    auto kfn = attn_simt::kernel<T>;
+    if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
+      return cuda_status(e);
+    ++g_launches;
+    prof_mark(st, true);
+    kfn<<<dim3(W, G), attn_simt::THREADS, sm, st>>>(aa, HG);
+    prof_mark(st, false);
+    if ((e = cudaGetLastError())) return cuda_status(e);
+    ++g_launches;
+    combine_kernel<T><<<dim3(2 * W, d.n_h), 128, 0, st>>>(aa);
+    if ((e = cudaGetLastError())) return cuda_status(e);
+  }
+  // (7) o_h = W_UV,h obar_h.
+  {
+    EpiStore<float> epi{out, (long long)d.n_h * d.d_v, d.d_v, 1.f};
+    if ((e = gemm<T>(at<T>(ws, P.obar), (long long)d.n_h * d.d_c, d.d_c, w->uv, d.d_c, (long long)d.d_v * d.d_c,
+                     R, d.d_v, d.d_c, d.n_h, epi, ws, P, st)))
+      return cuda_status(e);
+  }
+  return MLA_OK;
+}
+
+mla_status begin_call(void* ws, cudaStream_t st, const Plan& P) {
+  g_launches = 0;
+  return cuda_status(cudaMemsetAsync(ws, 0, P.partial, st));  // header + split-K counters
+}
+
+}  // namespace
+
+// =============================================================== C ABI ====
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_BOUNDS: return "MLA_ERR_DEVICE_BOUNDS";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int mla_last_launch_count(void) { return g_launches; }
+
+mla_status mla_profile_begin(int max_launches) {
+  if (max_launches <= 0 || g_prof.on) return MLA_ERR_INVALID_ARG;
+  g_prof.ev = static_cast<cudaEvent_t*>(calloc(2 * (size_t)max_launches, sizeof(cudaEvent_t)));
+  if (!g_prof.ev) return MLA_ERR_INVALID_ARG;
+  for (int i = 0; i < 2 * max_launches; ++i)
+    if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_prof.ev[j]);
+      free(g_prof.ev);
+      g_prof.ev = nullptr;
+      return MLA_ERR_CUDA;
+    }
+  g_prof.cap = max_launches;
+  g_prof.used = 0;
+  g_prof.on = true;
+  return MLA_OK;
+}
+
+mla_status mla_profile_end(double* total_ms, int* launches) {
+  if (!g_prof.on || !total_ms || !launches) return MLA_ERR_INVALID_ARG;
+  mla_status st = MLA_OK;
+  double sum = 0.0;
+  for (int i = 0; i < g_prof.used; ++i) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) {
+      st = MLA_ERR_CUDA;
+      break;
+    }
+    sum += ms;
+  }
+  *total_ms = sum;
+  *launches = g_prof.used;
+  for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+  free(g_prof.ev);
+  g_prof = Profiler{};
+  return st;
+}
+
+size_t mla_absorbed_weights_bytes(const mla_dims* dims) {
+  if (check_dims(dims) != MLA_OK) return 0;
+  return weight_layout(*dims).total;
+}
+
+mla_status mla_absorb_weights(const mla_dims* dims, const void* W_DKV, const void* W_KR, const void* W_DQ,
+                              const void* W_UQ, const void* W_QR, const void* W_UK, const void* W_UV,
+                              void* absorbed, size_t absorbed_bytes, mla_weights** out, cudaStream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if (!out || !W_DKV || !W_KR || !W_UQ || !W_QR || !W_UK || !W_UV || !absorbed) return MLA_ERR_INVALID_ARG;
+  if ((dims->d_cq > 0) != (W_DQ != nullptr)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(absorbed, 256)) return MLA_ERR_INVALID_ARG;
+  const mla_dims& d = *dims;
+  const WeightLayout L = weight_layout(d);
+  if (absorbed_bytes < L.total) return MLA_ERR_WORKSPACE;
+  const size_t e = esize(d);
+  char* base = static_cast<char*>(absorbed);
+  g_launches = 0;
+  cudaError_t err;
+  // Stacked [W_DKV; W_KR] and [W_UQ; W_QR]: plain contiguous copies.
+  size_t n1 = e * (size_t)d.d_c * d.d_model, n2 = e * (size_t)d.d_r * d.d_model;
+  if ((err = cudaMemcpyAsync(base + L.dkr, W_DKV, n1, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
+  if ((err = cudaMemcpyAsync(base + L.dkr + n1, W_KR, n2, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
+  if (d.d_cq > 0 &&
+      (err = cudaMemcpyAsync(base + L.dq, W_DQ, e * (size_t)d.d_cq * d.d_model, cudaMemcpyDeviceToDevice, stream)))
+    return cuda_status(err);
+  size_t q1 = e * (size_t)d.n_h * d.d_h * d_in(d), q2 = e * (size_t)d.n_h * d.d_r * d_in(d);
+  if ((err = cudaMemcpyAsync(base + L.uqr, W_UQ, q1, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
+  if ((err = cudaMemcpyAsync(base + L.uqr + q1, W_QR, q2, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
+  if ((err = cudaMemcpyAsync(base + L.uv, W_UV, e * (size_t)d.n_h * d.d_v * d.d_c, cudaMemcpyDeviceToDevice,
+                             stream)))
+    return cuda_status(err);
+  // Per-head transpose of W_UK: [n_h][d_h][d_c] -> [n_h][d_c][d_h].
+  {
+    dim3 grid(ceil_div(d.d_c, 32), ceil_div(d.d_h, 32), d.n_h);
+    ++g_launches;
+    if (d.dtype == MLA_BF16)
+      transpose_heads_kernel<__nv_bfloat16><<<grid, dim3(32, 8), 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(W_UK), reinterpret_cast<__nv_bfloat16*>(base + L.ukt), d.d_h, d.d_c);
+    else
+      transpose_heads_kernel<float><<<grid, dim3(32, 8), 0, stream>>>(
+          static_cast<const float*>(W_UK), reinterpret_cast<float*>(base + L.ukt), d.d_h, d.d_c);
+    if ((err = cudaGetLastError())) return cuda_status(err);
+  }
+  mla_weights* w = static_cast<mla_weights*>(calloc(1, sizeof(mla_weights)));
+  if (!w) return MLA_ERR_INVALID_ARG;
+  w->d = d;
+  w->scale = d.softmax_scale > 0.f ? d.softmax_scale : (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  w->esz = e;
+  w->dkr = base + L.dkr;
+  w->dq = d.d_cq > 0 ? base + L.dq : nullptr;
+  w->uqr = base + L.uqr;
+  w->ukt = base + L.ukt;
+  w->uv = base + L.uv;
+  for (int i = 0; i < d.d_r / 2; ++i) w->theta[i] = pow((double)d.rope_base, -2.0 * i / d.d_r);
+  *out = w;
+  return MLA_OK;
+}
+
+void mla_release_weights(mla_weights* w) { free(w); }
+
+mla_status mla_weights_dims(const mla_weights* w, mla_dims* dims) {
+  if (!w || !dims) return MLA_ERR_INVALID_ARG;
+  *dims = w->d;
+  return MLA_OK;
+}
+
+size_t mla_append_workspace_bytes(const mla_dims* dims, int T) {
+  if (check_dims(dims) != MLA_OK || T < 0) return 0;
+  return make_plan(*dims, T, false).total;
+}
+
+mla_status mla_append_latent(const mla_weights* w, const void* h, const int32_t* seq_idx, const int32_t* pos,
+                             const int32_t* page_table, int num_seqs, int max_pages, int num_pages, void* cache,
+                             int T, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || T < 0 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !seq_idx || !pos || !page_table || !cache || !workspace) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h, 16) || !aligned(cache, 16)) return MLA_ERR_INVALID_ARG;
+  const Plan P = make_plan(w->d, T, false);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  const int n_seq = num_seqs;
+  if (w->d.dtype == MLA_BF16)
+    return append_impl<__nv_bfloat16>(w, h, seq_idx, pos, 0, n_seq, page_table, max_pages, num_pages, cache, T,
+                                      workspace, P, stream);
+  return append_impl<float>(w, h, seq_idx, pos, 0, n_seq, page_table, max_pages, num_pages, cache, T, workspace,
+                            P, stream);
+}
+
+size_t mla_decode_workspace_bytes(const mla_dims* dims, int B, int n_q, int max_kv_len) {
+  if (check_dims(dims) != MLA_OK || B <= 0 || n_q <= 0 || max_kv_len < n_q) return 0;
+  return make_plan(*dims, B * n_q, true).total;
+}
+
+mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_len, const int32_t* page_table,
+                      int max_pages, int num_pages, const void* cache, float* out, int B, int n_q, int max_kv_len,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || B <= 0 || n_q <= 0 || max_kv_len < n_q || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!h_q || !kv_len || !page_table || !cache || !out || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)max_pages * w->d.page_size < max_kv_len) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h_q, 16) || !aligned(cache, 16) || !aligned(out, 16))
+    return MLA_ERR_INVALID_ARG;
+  const Plan P = make_plan(w->d, B * n_q, true);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  if (w->d.dtype == MLA_BF16)
+    return attend_impl<__nv_bfloat16>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out,
+                                      B * n_q, max_kv_len, workspace, P, stream);
+  return attend_impl<float>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out, B * n_q,
+                            max_kv_len, workspace, P, stream);
+}
+
+size_t mla_prefill_workspace_bytes(const mla_dims* dims, int B, int S) {
+  if (check_dims(dims) != MLA_OK || B <= 0 || S <= 0) return 0;
+  return make_plan(*dims, B * S, true).total;
+}
+
+mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_table, int max_pages,
+                       int num_pages, void* cache, float* out, int B, int S, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || B <= 0 || S <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!h || !page_table || !cache || !out || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)max_pages * w->d.page_size < S) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h, 16) || !aligned(cache, 16) || !aligned(out, 16))
+    return MLA_ERR_INVALID_ARG;
+  const Plan P = make_plan(w->d, B * S, true);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  if (w->d.dtype == MLA_BF16) {
+    s = append_impl<__nv_bfloat16>(w, h, nullptr, nullptr, S, B, page_table, max_pages, num_pages, cache, B * S,
+                                   workspace, P, stream);
+    if (s != MLA_OK) return s;
+    return attend_impl<__nv_bfloat16>(w, h, nullptr, S, S, S, page_table, max_pages, num_pages, cache, out, B * S,
+                                      S, workspace, P, stream);
+  }
+  s = append_impl<float>(w, h, nullptr, nullptr, S, B, page_table, max_pages, num_pages, cache, B * S, workspace,
+                         P, stream);
+  if (s != MLA_OK) return s;
+  return attend_impl<float>(w, h, nullptr, S, S, S, page_table, max_pages, num_pages, cache, out, B * S, S,
+                            workspace, P, stream);
+}
+
+mla_status mla_get_error(const void* workspace, cudaStream_t stream) {
+  if (!workspace) return MLA_ERR_INVALID_ARG;
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
+  if (word & kErrBounds) return MLA_ERR_DEVICE_BOUNDS;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+/*
+ * mla.h -- C ABI of libmla: multi-head latent attention computed on a paged,
+ * compressed latent cache, with weight absorption and decoupled RoPE, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (pages named by title and section):
+ *   - "ai-decoupled-rope-mla" (operatorworld), decoupled-RoPE section: each
+ *     token caches a latent c_t = W_DKV h_t and a small position key
+ *     k_R,t = RoPE_t(W_KR h_t); the query has a content part q_C and a rotated
+ *     position part q_R; the score adds a content term and a position term.
+ *   - "Latent Attention Meets RoPE" (sahipadhai), "Two small, telling details":
+ *     the position key is one vector shared by all heads, and only the latent
+ *     and that key are cached.
+ *   - "ai-decoupled-rope-mla", absorption equations: q~ = W_UK^T q_C scores the
+ *     latent directly, and the output is W_UV applied to sum_t alpha_t c_t.
+ *   - "Detailed Illustration of the Problem" (notion), Step 1: an optional
+ *     query latent c_Q = W_DQ h feeds the query projections.
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers owned by the caller, dense,
+ *     row-major, with the element type given by mla_dims.dtype (fp32 or
+ *     bf16) unless stated otherwise.  Index arrays are int32.
+ *   - Every call is asynchronous on `stream`.  Argument errors are reported
+ *     before anything is launched.  Errors found on the device (a page id out
+ *     of range, a length out of range) are OR-ed into an error word at the
+ *     start of the caller's workspace and never trap; mla_get_error reads it.
+ *   - The library allocates no device memory.  Scratch space is the caller's
+ *     `workspace`, sized by the *_workspace_bytes queries; the workspace of a
+ *     call must not be used by another call that may run at the same time.
+ *   - Cache layout: [num_pages, page_size, d_c + d_r]; row (page p, slot s)
+ *     holds [c_t (d_c) | k_R,t (d_r)] for the token whose position is
+ *     j*page_size + s, where page_table[seq*max_pages + j] == p.
+ *   - Weight orientation is column-vector, y = W x: W_DKV [d_c, d_model],
+ *     W_KR [d_r, d_model], W_DQ [d_cq, d_model], W_UQ [n_h*d_h, d_in],
+ *     W_QR [n_h*d_r, d_in], W_UK [n_h*d_h, d_c], W_UV [n_h*d_v, d_c], where
+ *     d_in = d_cq when d_cq > 0, else d_model.  Rows h*d_h .. h*d_h+d_h-1 of
+ *     W_UK (and likewise W_UQ, W_QR, W_UV) belong to head h.
+ *   - RoPE rotates interleaved pairs (2i, 2i+1) by pos * rope_base^(-2i/d_r);
+ *     the pages print only the rotation family, so the frequencies and the
+ *     pairing are the reading this library takes.
+ *   - A query at position m attends to the keys at positions 0..m, itself
+ *     included (new tokens are appended before they attend).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,    /* null pointer, bad size, misaligned buffer   */
+  MLA_ERR_UNSUPPORTED = -2,    /* dimensions this build has no kernel for     */
+  MLA_ERR_WORKSPACE = -3,      /* workspace or weight buffer too small        */
+  MLA_ERR_CUDA = -4,           /* a CUDA runtime call failed                  */
+  MLA_ERR_DEVICE_BOUNDS = -5,  /* device-side check: index out of range       */
+  MLA_ERR_TIMEOUT = -6         /* device-side bounded wait gave up            */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+typedef struct {
+  int n_h;              /* query heads                                       */
+  int d_h;              /* per-head content query/key width                  */
+  int d_v;              /* per-head value width                              */
+  int d_c;              /* KV latent width                                   */
+  int d_r;              /* shared RoPE key width (even)                      */
+  int d_model;          /* hidden width                                      */
+  int d_cq;             /* query latent width; 0 = no query latent           */
+  float rope_base;      /* e.g. 10000                                        */
+  float softmax_scale;  /* 0 selects 1/sqrt(d_h + d_r) on both score terms   */
+  int page_size;        /* tokens per cache page; this build supports 64     */
+  mla_dtype dtype;      /* element type of weights, hidden states and cache  */
+} mla_dims;
+
+/* Opaque host-side handle created by mla_absorb_weights.  It holds the
+ * dimensions and pointers into the caller's `absorbed` device buffer. */
+typedef struct mla_weights mla_weights;
+
+/* ---------------------------------------------------------------------------
+ * Weights.  Absorption (the decoupled-RoPE page's absorption equations) is
+ * independent of the cache, so the weight-side layouts are prepared once:
+ * W_DKV and W_KR stacked into one [d_c + d_r, d_model] matrix, W_UQ and W_QR
+ * stacked into one [n_h*(d_h + d_r), d_in] matrix, each head's W_UK slice
+ * transposed to [d_c, d_h], and W_UV and W_DQ copied.  The products with W_UK
+ * and W_UV are taken at run time on the query side and after the latent sum.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device memory mla_absorb_weights needs in `absorbed`; 0 if the
+ * dimensions are invalid or unsupported. */
+size_t mla_absorbed_weights_bytes(const mla_dims* dims);
+
+/* Copies and re-lays-out the weights into `absorbed` (device, caller-owned,
+ * at least mla_absorbed_weights_bytes(dims) bytes, 256-byte aligned) and
+ * returns a handle in *out.  W_DQ must be NULL iff dims->d_cq == 0.  The input
+ * weights may be freed once the stream has passed this call; `absorbed` must
+ * outlive the handle.  Errors: MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED,
+ * MLA_ERR_WORKSPACE (buffer too small), MLA_ERR_CUDA. */
+mla_status mla_absorb_weights(const mla_dims* dims, const void* W_DKV, const void* W_KR,
+                              const void* W_DQ, const void* W_UQ, const void* W_QR,
+                              const void* W_UK, const void* W_UV, void* absorbed,
+                              size_t absorbed_bytes, mla_weights** out, cudaStream_t stream);
+
+/* Frees the host-side handle (not the caller's device buffer). NULL is a no-op. */
+void mla_release_weights(mla_weights* w);
+
+/* Copies the handle's dimensions into *dims. */
+mla_status mla_weights_dims(const mla_weights* w, mla_dims* dims);
+
+/* ---------------------------------------------------------------------------
+ * Append.  For T tokens with hidden states h [T, d_model], sequence index
+ * seq_idx[T] and position pos[T], computes c = W_DKV h and
+ * k_R = RoPE_pos(W_KR h) (decoupled-RoPE page; the shared position key of
+ * "Latent Attention Meets RoPE") with fp32 accumulation and writes
+ * [c | k_R] (rounded to the cache type) into the cache row for (seq, pos).
+ * page_table is [num_seqs, max_pages]; a seq_idx outside [0, num_seqs), a
+ * position outside [0, max_pages*page_size) or a page id outside
+ * [0, num_pages) sets MLA_ERR_DEVICE_BOUNDS in the workspace error word and
+ * skips that token's write.
+ * Workspace: mla_append_workspace_bytes(dims, T).
+ * ------------------------------------------------------------------------- */
+size_t mla_append_workspace_bytes(const mla_dims* dims, int T);
+mla_status mla_append_latent(const mla_weights* w, const void* h, const int32_t* seq_idx,
+                             const int32_t* pos, const int32_t* page_table, int num_seqs,
+                             int max_pages, int num_pages, void* cache, int T, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Decode.  B sequences each with n_q new tokens whose hidden states are
+ * h_q [B, n_q, d_model]; kv_len[b] (device) counts the keys of sequence b
+ * including its n_q new tokens, which must already be appended
+ * (mla_append_latent) at positions kv_len[b]-n_q .. kv_len[b]-1.  New token q
+ * of sequence b sits at position kv_len[b]-n_q+q and attends to keys
+ * 0 .. kv_len[b]-n_q+q.  Writes out [B, n_q, n_h, d_v] as fp32:
+ *   q_C, q_R from h (through c_Q = W_DQ h when d_cq > 0),
+ *   q~_h = W_UK,h^T q_C,h,  a_t = s*(q~_h . c_t) + s*(RoPE_m(q_R,h) . k_R,t),
+ *   alpha = softmax(a),     o_h = W_UV,h sum_t alpha_t c_t.
+ * max_kv_len bounds kv_len (host value used for workspace sizing); kv_len[b]
+ * outside [n_q, max_kv_len] sets MLA_ERR_DEVICE_BOUNDS and that sequence's
+ * outputs are unspecified.  Workspace: mla_decode_workspace_bytes(...).
+ * ------------------------------------------------------------------------- */
+size_t mla_decode_workspace_bytes(const mla_dims* dims, int B, int n_q, int max_kv_len);
+mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_len,
+                      const int32_t* page_table, int max_pages, int num_pages, const void* cache,
+                      float* out, int B, int n_q, int max_kv_len, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Causal prefill on the absorbed path.  h [B, S, d_model]: token s of
+ * sequence b sits at position s.  Appends all B*S tokens to the cache (the
+ * page table must cover S positions per sequence), then every token attends
+ * to positions <= its own.  Writes out [B, S, n_h, d_v] fp32.
+ * Workspace: mla_prefill_workspace_bytes(dims, B, S).
+ * ------------------------------------------------------------------------- */
+size_t mla_prefill_workspace_bytes(const mla_dims* dims, int B, int S);
+mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_table,
+                       int max_pages, int num_pages, void* cache, float* out, int B, int S,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Status.
+ * ------------------------------------------------------------------------- */
+/* Waits for `stream`, then returns the error recorded on the device by the
+ * most recent call that used `workspace` (MLA_OK if none). */
+mla_status mla_get_error(const void* workspace, cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* mla_status_string(mla_status s);
+
+/* Number of kernel launches the most recent call on this host thread issued
+ * (for launch accounting in benchmarks). */
+int mla_last_launch_count(void);
+
+/* Kernel timing for benchmarks.  Between mla_profile_begin and
+ * mla_profile_end, every launch of the latent-attention kernel (the step that
+ * streams the cache) made on this host thread is bracketed by a pair of CUDA
+ * events recorded on the call's stream; at most max_launches launches are
+ * timed.  mla_profile_end waits for the last event and returns the summed
+ * kernel time in milliseconds and the number of timed launches.  Creates CUDA
+ * events (no device memory).  Errors: MLA_ERR_INVALID_ARG, MLA_ERR_CUDA. */
+mla_status mla_profile_begin(int max_launches);
+mla_status mla_profile_end(double* total_ms, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

@@ -189,15 +189,16 @@ def attend_materialised(dims: Dims, w: Weights, q_c, q_r, c, k_r, q_pos, k_pos,
     k_pos = np.asarray(k_pos)
     visible = k_pos[None, :] <= q_pos[:, None]                    # [Q, T]
     out = np.empty((q_c.shape[0], n_h, d_v))
-    pos_term = np.einsum("qhr,tr->qht", q_r, k_r)                 # [Q, n_h, T]
+    pos_term = np.matmul(q_r, k_r.T)                              # [Q, n_h, T]
     for h0 in range(0, n_h, head_chunk):
         hs = slice(h0, min(n_h, h0 + head_chunk))
-        k_c = np.einsum("hdc,tc->htd", W_UK[hs], c)               # [h, T, d_h]
-        v = np.einsum("hvc,tc->htv", W_UV[hs], c)                 # [h, T, d_v]
-        a = (np.einsum("qhd,htd->qht", q_c[:, hs], k_c) + pos_term[:, hs]) * scale
+        k_c = np.matmul(c[None], W_UK[hs].transpose(0, 2, 1))     # [h, T, d_h]  (K_C = W_UK,h c_t)
+        v = np.matmul(c[None], W_UV[hs].transpose(0, 2, 1))       # [h, T, d_v]  (V = W_UV,h c_t)
+        content = np.matmul(q_c[:, hs].transpose(1, 0, 2), k_c.transpose(0, 2, 1))  # [h, Q, T]
+        a = (content.transpose(1, 0, 2) + pos_term[:, hs]) * scale
         a = np.where(visible[:, None, :], a, -np.inf)
-        alpha = _softmax(a)
-        out[:, hs] = np.einsum("qht,htv->qhv", alpha, v)
+        alpha = _softmax(a)                                       # [Q, h, T]
+        out[:, hs] = np.matmul(alpha.transpose(1, 0, 2), v).transpose(1, 0, 2)
     return out
 
 
