@@ -8,6 +8,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
@@ -142,7 +144,7 @@ mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
 template <typename T, class Epi>
 cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                  int M, int N, int K, int batch, const Epi& epi, void* ws, const Plan& P,
-                 cudaStream_t st) {
+                 cudaStream_t st, int tile_split_cap = kSplitKTileSplits) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   GemmArgs a{};
   a.A = A; a.lda = lda; a.strideA = sA;
@@ -154,7 +156,7 @@ cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long
   if (tiles < want && tiles <= kCounterCap) {
     splits = ceil_div(want, tiles);
     splits = std::min(splits, std::max(1, K / 256));
-    splits = std::min(splits, kSplitKTileSplits / tiles);
+    splits = std::min(splits, tile_split_cap / tiles);
     splits = std::max(splits, 1);
   }
   int kchunk = ceil_div(ceil_div(K, splits), 32) * 32;
@@ -514,3 +516,108 @@ mla_status mla_get_error(const void* workspace, cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ===================================================================
+// Append without a caller workspace.
+//
+// Some callers cannot hand this library a workspace because they cannot
+// allocate device memory at the point where they append: an inference engine
+// that owns every byte of HBM through its own fixed pool and forbids other
+// allocations, code running while a CUDA graph is being captured (where
+// cudaMalloc is not permitted), or a host thread that must not take the
+// implicit device synchronisation cudaMalloc/cudaFree can cause.  For them,
+// mla_append_latent_noalloc keeps the append's scratch (the split-K partial
+// tiles and their arrival counters) in one fixed array in this library's own
+// device memory instead.
+//
+// The array is a file-scope __device__ variable, so every GPU that loads
+// libmla holds it (kNoAllocScratchBytes, about 2 MiB) until the process exits.
+// Host code must not pass the symbol itself to a kernel (on the host it is
+// only a stand-in, not a device address); its device address is looked up
+// once per device with cudaGetSymbolAddress and cached.
+// ===================================================================
+namespace {
+
+constexpr int kNoAllocMaxT = 256;                 // tokens per call
+constexpr int kNoAllocTileSplits = 128;           // split-K tiles x splits
+constexpr size_t kNoAllocHdr = 256;               // unused error word slot
+constexpr size_t kNoAllocCounters = sizeof(int) * kCounterCap;
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocHdr + kNoAllocCounters + sizeof(float) * (size_t)kNoAllocTileSplits * 64 * 64;
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::once_flag g_noalloc_once[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on
+// the first call made with that device current).
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = (g_noalloc_err[dev] == cudaSuccess) ? p : nullptr;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess) return g_noalloc_err[dev];
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+template <typename T>
+mla_status append_noalloc_impl(const mla_weights* w, const void* h, const int32_t* seq_idx, const int32_t* pos,
+                               const int32_t* page_table, int num_seqs, int max_pages, int num_pages, void* cache,
+                               int T_, int32_t* device_error, void* scratch, cudaStream_t st) {
+  const mla_dims& d = w->d;
+  Plan P{};
+  P.hdr = 0;
+  P.counters = kNoAllocHdr;
+  P.partial = kNoAllocHdr + kNoAllocCounters;
+  P.total = kNoAllocScratchBytes;
+  EpiAppend<T> epi{};
+  epi.cache = static_cast<T*>(cache);
+  epi.seq_idx = seq_idx;
+  epi.pos = pos;
+  epi.prefill_S = 0;
+  epi.page_table = page_table;
+  for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
+  epi.max_pages = max_pages;
+  epi.num_pages = num_pages;
+  epi.page_size = d.page_size;
+  epi.d_c = d.d_c;
+  epi.d_cr = d.d_c + d.d_r;
+  epi.n_seq = num_seqs;
+  epi.err = device_error ? reinterpret_cast<int*>(device_error) : at<int>(scratch, P.hdr);
+  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, d.d_c + d.d_r, d.d_model, 1, epi, scratch,
+                             P, st, kNoAllocTileSplits));
+}
+
+}  // namespace
+
+extern "C" mla_status mla_append_latent_noalloc(const mla_weights* w, const void* h, const int32_t* seq_idx,
+                                                const int32_t* pos, const int32_t* page_table, int num_seqs,
+                                                int max_pages, int num_pages, void* cache, int T,
+                                                int32_t* device_error, cudaStream_t stream) {
+  if (!w || T < 0 || num_seqs <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (T > kNoAllocMaxT) return MLA_ERR_WORKSPACE;
+  if (T == 0) return MLA_OK;
+  if (!h || !seq_idx || !pos || !page_table || !cache) return MLA_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(cache, 16) || (device_error && !aligned(device_error, 4)))
+    return MLA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return MLA_ERR_CUDA;
+  g_launches = 0;
+  // The arrival counters must start at zero; the array keeps whatever the
+  // previous call left in it.
+  if (cudaMemsetAsync(scratch, 0, kNoAllocHdr + kNoAllocCounters, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  if (w->d.dtype == MLA_BF16)
+    return append_noalloc_impl<__nv_bfloat16>(w, h, seq_idx, pos, page_table, num_seqs, max_pages, num_pages,
+                                              cache, T, device_error, scratch, stream);
+  return append_noalloc_impl<float>(w, h, seq_idx, pos, page_table, num_seqs, max_pages, num_pages, cache, T,
+                                    device_error, scratch, stream);
+}

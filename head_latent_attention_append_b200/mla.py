@@ -24,8 +24,9 @@ EXPORTED = [
     "mla_absorbed_weights_bytes", "mla_absorb_weights", "mla_release_weights", "mla_weights_dims",
     "mla_append_workspace_bytes", "mla_append_latent", "mla_decode_workspace_bytes", "mla_decode",
     "mla_prefill_workspace_bytes", "mla_prefill", "mla_get_error", "mla_status_string",
-    "mla_last_launch_count", "mla_profile_begin", "mla_profile_end",
+    "mla_last_launch_count", "mla_profile_begin", "mla_profile_end", "mla_append_latent_noalloc",
 ]
+APPEND_NOALLOC_MAX_T = 256
 
 
 class MlaError(RuntimeError):
@@ -67,6 +68,7 @@ def _load():
         "mla_status_string": (ctypes.c_char_p, [S]),
         "mla_last_launch_count": (I, []),
         "mla_profile_begin": (S, [I]),
+        "mla_append_latent_noalloc": (S, [P, P, P, P, P, I, I, I, P, I, P, P]),
         "mla_profile_end": (S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
     }
     for name, (res, args) in sig.items():
@@ -162,6 +164,16 @@ def append_latent(w: Weights, h, seq_idx, pos, page_table, num_pages: int, cache
     _check("mla_append_latent", lib.mla_append_latent(
         w.handle, _ptr(h), _ptr(seq_idx), _ptr(pos), _ptr(page_table), num_seqs, max_pages, num_pages,
         _ptr(cache), T, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def append_latent_noalloc(w: Weights, h, seq_idx, pos, page_table, num_pages: int, cache, device_error=None,
+                          stream=None):
+    """mla_append_latent without a workspace (scratch inside libmla; T <= 256)."""
+    T = h.shape[0]
+    num_seqs, max_pages = page_table.shape
+    _check("mla_append_latent_noalloc", lib.mla_append_latent_noalloc(
+        w.handle, _ptr(h), _ptr(seq_idx), _ptr(pos), _ptr(page_table), num_seqs, max_pages, num_pages,
+        _ptr(cache), T, _ptr(device_error), _stream(stream)))
 
 
 def decode(w: Weights, h_q, kv_len, page_table, num_pages: int, cache, out, max_kv_len: int, workspace,

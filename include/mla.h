@@ -130,6 +130,31 @@ mla_status mla_append_latent(const mla_weights* w, const void* h, const int32_t*
                              int max_pages, int num_pages, void* cache, int T, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream);
 
+/* Append without a workspace.  The pages have no counterpart to this entry
+ * point; it exists for callers that cannot allocate device memory where they
+ * append (an engine that owns all of HBM through its own pool, code running
+ * under CUDA stream capture, a thread that must not take cudaMalloc's implicit
+ * synchronisation).  Same computation and arguments as mla_append_latent,
+ * except that the scratch lives in a fixed array inside libmla's own device
+ * memory (about 2 MiB, held on every GPU that loads the library until the
+ * process exits) and T is limited to MLA_APPEND_NOALLOC_MAX_T tokens; a larger
+ * T returns MLA_ERR_WORKSPACE.  It calls no allocating function.
+ *   - device_error: optional device int32 (NULL to ignore) into which
+ *     MLA_ERR_DEVICE_BOUNDS conditions are OR-ed as the value 1; the caller zeroes
+ *     it.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and re-zeroes the parts that must start
+ *     at zero; calls that can overlap on the GPU (different streams, or
+ *     different host threads on one device) race on it and must be serialised
+ *     by the caller. */
+#define MLA_APPEND_NOALLOC_MAX_T 256
+mla_status mla_append_latent_noalloc(const mla_weights* w, const void* h, const int32_t* seq_idx,
+                                     const int32_t* pos, const int32_t* page_table, int num_seqs,
+                                     int max_pages, int num_pages, void* cache, int T,
+                                     int32_t* device_error, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Decode.  B sequences each with n_q new tokens whose hidden states are
  * h_q [B, n_q, d_model]; kv_len[b] (device) counts the keys of sequence b
