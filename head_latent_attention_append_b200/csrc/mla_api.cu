@@ -10,7 +10,10 @@
 
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "prep.cuh"
@@ -71,10 +74,11 @@ mla_status check_dims(const mla_dims* d) {
   if (d->page_size != 64) return MLA_ERR_UNSUPPORTED;
   if (d->n_h > 128) return MLA_ERR_UNSUPPORTED;
   if (d->dtype == MLA_BF16) {
-    // 16-byte row alignment for the tensor-core loads; d_c split evenly.
-    if (d->d_h % 8 || d->d_v % 8 || d->d_c % 64 || d->d_r % 16 || d->d_model % 8 || d->d_cq % 8)
+    // 16-byte row alignment for the tensor-core loads; the latent splits into
+    // two halves of whole 64-column chunks; a cache row is at most nine chunks.
+    if (d->d_h % 8 || d->d_v % 8 || d->d_c % 128 || d->d_r % 16 || d->d_model % 8 || d->d_cq % 8)
       return MLA_ERR_UNSUPPORTED;
-    if (d->d_c > 512) return MLA_ERR_UNSUPPORTED;
+    if (d->d_c > 512 || d->d_c + d->d_r > 576) return MLA_ERR_UNSUPPORTED;
   } else {
     if (d->d_c > 512) return MLA_ERR_UNSUPPORTED;
   }
@@ -139,6 +143,37 @@ T* at(void* base, size_t off) {
 }
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda at build time).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D view of the page pool: rows = num_pages * page_size tokens, columns =
+// d_c + d_r bf16; boxes of 64 tokens x 64 columns, 128-byte swizzle.
+// Columns past d_c + d_r read as zero.
+bool encode_cache_map(CUtensorMap* map, const void* cache, int d_cr, long long rows) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)d_cr, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)d_cr * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(cache), gdim, gstride, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 // ----------------------------------------------------------- GEMM launcher
 template <typename T, class Epi>
@@ -257,11 +292,14 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   aa.obar = at<T>(ws, P.obar);
   aa.err = err;
 
-  // Heads per CTA: a power of two so that 256 threads split evenly.
+  constexpr bool kTensorCores = sizeof(T) == 2;
+  // fp32: heads per CTA a power of two so that 256 threads split evenly.
   int HG = 16;
   while (HG > d.n_h) HG >>= 1;
-  const int G = ceil_div(d.n_h, HG);
-  int W = std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
+  const int G = kTensorCores ? 2 : ceil_div(d.n_h, HG);
+  // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
+  int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
+                       : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
   {
     SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
     ++g_launches;
@@ -269,7 +307,19 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (5) attention on the latent cache, (6) combine of split row blocks.
-  {
+  if constexpr (kTensorCores) {
+    CUtensorMap map;
+    if (!encode_cache_map(&map, cache, d_cr, (long long)num_pages * d.page_size)) return MLA_ERR_CUDA;
+    attn_tc::Params pp{aa, ceil_div(d_cr, 64), d.d_c / 2};
+    if ((e = cudaFuncSetAttribute(attn_tc::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)attn_tc::SMEM_BYTES)))
+      return cuda_status(e);
+    ++g_launches;
+    prof_mark(st, true);
+    attn_tc::kernel<<<dim3(W, 2), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
+    prof_mark(st, false);
+    if ((e = cudaGetLastError())) return cuda_status(e);
+  } else {
     size_t sm = attn_simt::smem_bytes(HG, d_cr);
     auto kfn = attn_simt::kernel<T>;
     if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
@@ -279,6 +329,8 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     kfn<<<dim3(W, G), attn_simt::THREADS, sm, st>>>(aa, HG);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
+  }
+  {
     ++g_launches;
     combine_kernel<T><<<dim3(2 * W, d.n_h), 128, 0, st>>>(aa);
     if ((e = cudaGetLastError())) return cuda_status(e);
