@@ -37,7 +37,7 @@ namespace attn_simt {
 constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
 
 template <typename T>
-__global__ void __launch_bounds__(THREADS) kernel(AttnArgs a, int HG) {
+__global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) {
   extern __shared__ float smem[];
   const int pitch = a.d_cr + 1;
   float* Qs = smem;                    // [HG][pitch]

@@ -26,9 +26,11 @@
 // the P*V MMA is done.  The two CTAs of a pair read the same pages at about
 // the same time, so the second read is served by L2.
 //
-// Warp roles (256 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 =
-// MMA issuer, warp 2 = TMEM allocator, warps 4-7 = softmax / epilogue (thread
-// r owns row r = TMEM lane r).  Every wait is bounded (sm100::mbar_wait).
+// Warp roles (256 threads): warps 0 and 3 = TMA producers (one per ring),
+// warp 1 = MMA issuer (each runs warp-uniformly; one elected lane issues),
+// warp 2 = TMEM allocator,
+// warps 4-7 = softmax / epilogue (thread r owns row r = TMEM lane r).  Every
+// wait is bounded (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -71,7 +73,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b, float& sum) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -126,9 +128,13 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (tid == 0) {
-    // ------------------------------------------------------ TMA producer
-    uint32_t a_cnt = 0, b_cnt = 0;
+  if (warp == 0 || warp == 3) {
+    // ----------------------------------------------------- TMA producers
+    // Warp 0 feeds the score-only ring, warp 3 the own-half ring; each walks
+    // every tile of the worker on its own, so neither ring waits for the
+    // other's slots.  The warp runs uniformly; one elected lane issues.
+    const bool ring_b = (warp == 3);
+    uint32_t cnt = 0;  // chunks (score-only ring) or tile groups (own-half ring) issued
     bool ok = true;
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const Seg g = segs[si];
@@ -136,43 +142,53 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUt
       for (int t = g.t_lo; t < g.t_hi && ok; ++t) {
         int page = a.page_table[(long long)seq * a.max_pages + t];
         if (page < 0 || page >= a.num_pages) {
-          flag_error(a.err, kErrBounds);
+          if (!ring_b && elect_one()) flag_error(a.err, kErrBounds);
           page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
         }
         const int y = page * KT;
-        const uint32_t gs = b_cnt % B_GROUPS;
-        for (int c = 0; c < nkc; ++c) {
-          if (c >= own0 && c < own0 + npv) {
-            if (c == own0) {
-              if (!(ok = mbar_wait(&b_empty[gs], ((b_cnt / B_GROUPS) & 1) ^ 1, abort_flag, a.err))) break;
-              mbar_arrive_expect_tx(&b_full[gs], npv * CHUNK_BYTES);
+        if (ring_b) {
+          const uint32_t gs = cnt % B_GROUPS;
+          if (!(ok = mbar_wait_warp(&b_empty[gs], ((cnt / B_GROUPS) & 1) ^ 1, abort_flag, a.err))) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&b_full[gs], npv * CHUNK_BYTES);
+            for (int q = 0; q < npv; ++q)
+              tma_load_2d(smem + OFF_B + gs * B_GROUP_BYTES + q * CHUNK_BYTES, &tmap, (own0 + q) * 64, y,
+                          &b_full[gs]);
+          }
+          __syncwarp();
+          ++cnt;
+        } else {
+          for (int c = 0; c < nkc; ++c) {
+            if (c >= own0 && c < own0 + npv) continue;
+            const uint32_t slot = cnt % A_SLOTS;
+            if (!(ok = mbar_wait_warp(&a_empty[slot], ((cnt / A_SLOTS) & 1) ^ 1, abort_flag, a.err))) break;
+            if (elect_one()) {
+              mbar_arrive_expect_tx(&a_full[slot], CHUNK_BYTES);
+              tma_load_2d(smem + OFF_A + slot * CHUNK_BYTES, &tmap, c * 64, y, &a_full[slot]);
             }
-            tma_load_2d(smem + OFF_B + gs * B_GROUP_BYTES + (c - own0) * CHUNK_BYTES, &tmap, c * 64, y,
-                        &b_full[gs]);
-          } else {
-            const uint32_t slot = a_cnt % A_SLOTS;
-            if (!(ok = mbar_wait(&a_empty[slot], ((a_cnt / A_SLOTS) & 1) ^ 1, abort_flag, a.err))) break;
-            mbar_arrive_expect_tx(&a_full[slot], CHUNK_BYTES);
-            tma_load_2d(smem + OFF_A + slot * CHUNK_BYTES, &tmap, c * 64, y, &a_full[slot]);
-            ++a_cnt;
+            __syncwarp();
+            ++cnt;
           }
         }
-        ++b_cnt;
       }
     }
     if (*abort_flag) {
       // Let every copy already issued land before the CTA can exit.
-      for (uint32_t s = 0; s < A_SLOTS && s < a_cnt; ++s) {
-        uint32_t last = ((a_cnt - 1 - s) / A_SLOTS) * A_SLOTS + s;
-        mbar_wait(&a_full[s], (last / A_SLOTS) & 1, abort_flag, nullptr, 50000000ull, false);
-      }
-      for (uint32_t s = 0; s < B_GROUPS && s < b_cnt; ++s) {
-        uint32_t last = ((b_cnt - 1 - s) / B_GROUPS) * B_GROUPS + s;
-        mbar_wait(&b_full[s], (last / B_GROUPS) & 1, abort_flag, nullptr, 50000000ull, false);
+      const uint32_t n = ring_b ? B_GROUPS : A_SLOTS;
+      uint64_t* full = ring_b ? b_full : a_full;
+      for (uint32_t q = 0; q < n && q < cnt; ++q) {
+        const uint32_t last = q + n * ((cnt - 1 - q) / n);
+        mbar_wait_warp(&full[q], (last / n) & 1, abort_flag, nullptr, 50000000ull, false);
       }
     }
-  } else if (tid == 32) {
+  } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
+    // Issue order per tile: the score MMA of tile t (own-half chunks first,
+    // they were prefetched furthest ahead), and the P*V MMA of tile t-1 as
+    // soon as its P is ready -- polled while waiting for score data, so a
+    // late chunk never holds back the release of the own-half ring.  The
+    // whole warp runs this loop with uniform values; one elected lane issues
+    // each tcgen05 instruction.
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);
     const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
     const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q;
@@ -180,72 +196,132 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUt
     const uint32_t sQ = smem_u32(smem + OFF_Q), sP = smem_u32(smem + OFF_P);
     uint32_t a_cnt = 0, b_cnt = 0, tg = 0, seg_k = 0;
     bool ok = true;
-    auto issue_pv = [&](uint32_t gs, uint32_t tile_tg, bool first) -> bool {
-      if (!mbar_wait(p_ready, tile_tg & 1, abort_flag, a.err)) return false;
-      if (first && seg_k > 0 && !mbar_wait(o_free, (seg_k - 1) & 1, abort_flag, a.err)) return false;
+    bool pv_pending = false, pv_first = false;
+    uint32_t pv_gs = 0, pv_tg = 0, pv_seg = 0;
+    // Issues the pending P*V MMA if its inputs are ready; never blocks.
+    auto try_pv = [&]() {
+      if (!pv_pending || !mbar_try_wait_warp(p_ready, pv_tg & 1)) return;
+      if (pv_first && pv_seg > 0 && !mbar_try_wait_warp(o_free, (pv_seg - 1) & 1)) return;
       tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < KT / 16; ++kk) {
-        const uint64_t ad = sdesc_sw128(sP + kk * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sB + gs * B_GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024);
-        mma_ss(tO, ad, bd, idPV, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sP + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sB + pv_gs * B_GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024);
+          mma_ss(tO, ad, bd, idPV, (pv_first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(pv_done);
+        tc_commit(&b_empty[pv_gs]);
       }
-      tc_commit(pv_done);
-      tc_commit(&b_empty[gs]);
+      __syncwarp();
+      pv_pending = false;
+    };
+    // Bounded wait on `bar` that keeps issuing the pending P*V meanwhile.
+    auto wait_polling = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait_warp(bar, parity)) {
+        try_pv();
+        int stop = 0;
+        if (*abort_flag) stop = 1;
+        else if (globaltimer_ns() - t0 > 2000000000ull) stop = 2;
+        stop = __shfl_sync(0xffffffffu, stop, 0);
+        if (stop) {
+          if (stop == 2 && elect_one()) {
+            *abort_flag = 1;
+            flag_error(a.err, kErrTimeout);
+          }
+          __syncwarp();
+          return false;
+        }
+      }
+      return true;
+    };
+    auto flush_pv = [&]() -> bool {
+      const uint64_t t0 = globaltimer_ns();
+      while (pv_pending) {
+        try_pv();
+        if (!pv_pending) break;
+        int stop = 0;
+        if (*abort_flag) stop = 1;
+        else if (globaltimer_ns() - t0 > 2000000000ull) stop = 2;
+        stop = __shfl_sync(0xffffffffu, stop, 0);
+        if (stop) {
+          if (stop == 2 && elect_one()) {
+            *abort_flag = 1;
+            flag_error(a.err, kErrTimeout);
+          }
+          __syncwarp();
+          return false;
+        }
+      }
       return true;
     };
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const Seg g = segs[si];
       const int n = g.t_hi - g.t_lo;
-      if (!(ok = mbar_wait(q_ready, seg_k & 1, abort_flag, a.err))) break;
+      if (!(ok = wait_polling(q_ready, seg_k & 1))) break;
       tc_fence_after();
-      uint32_t prev_gs = 0, prev_tg = 0;
       for (int i = 0; i < n && ok; ++i) {
-        if (tg > 0 && !(ok = mbar_wait(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
+        if (tg > 0 && !(ok = wait_polling(s_free, (tg - 1) & 1))) break;
         tc_fence_after();
         const uint32_t gs = b_cnt % B_GROUPS;
         uint32_t acc = 0;
-        for (int c = 0; c < nkc; ++c) {
-          const bool own = (c >= own0 && c < own0 + npv);
+        for (int k2 = 0; k2 < nkc; ++k2) {
+          // own-half chunks first, then the rest in column order
+          int c;
+          if (k2 < npv) c = own0 + k2;
+          else {
+            const int j = k2 - npv;
+            c = (j < own0) ? j : j + npv;
+          }
+          const bool own = k2 < npv;
           uint32_t bsrc, slot = 0;
           if (own) {
-            if (c == own0 && !(ok = mbar_wait(&b_full[gs], (b_cnt / B_GROUPS) & 1, abort_flag, a.err))) break;
-            bsrc = sB + gs * B_GROUP_BYTES + (c - own0) * CHUNK_BYTES;
+            if (k2 == 0 && !(ok = wait_polling(&b_full[gs], (b_cnt / B_GROUPS) & 1))) break;
+            bsrc = sB + gs * B_GROUP_BYTES + k2 * CHUNK_BYTES;
           } else {
             slot = a_cnt % A_SLOTS;
-            if (!(ok = mbar_wait(&a_full[slot], (a_cnt / A_SLOTS) & 1, abort_flag, a.err))) break;
+            if (!(ok = wait_polling(&a_full[slot], (a_cnt / A_SLOTS) & 1))) break;
             bsrc = sA + slot * CHUNK_BYTES;
           }
           tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bd = sdesc_sw128(bsrc + k * 32, 16, 1024);
+          if (elect_one()) {
             if (c < Q_TMEM_CHUNKS) {
-              mma_ts(tS, tQ + c * 32 + k * 8, bd, idS, acc);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_ts(tS, tQ + c * 32 + k * 8, sdesc_sw128(bsrc + k * 32, 16, 1024), idS, (acc | k) ? 1u : 0u);
             } else {
-              const uint64_t ad = sdesc_sw128(sQ + (c - Q_TMEM_CHUNKS) * Q_CHUNK_BYTES + k * 32, 16, 1024);
-              mma_ss(tS, ad, bd, idS, acc);
+              const uint32_t qa = sQ + (c - Q_TMEM_CHUNKS) * Q_CHUNK_BYTES;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_ss(tS, sdesc_sw128(qa + k * 32, 16, 1024), sdesc_sw128(bsrc + k * 32, 16, 1024), idS,
+                       (acc | k) ? 1u : 0u);
             }
-            acc = 1;
+            if (!own) tc_commit(&a_empty[slot]);
           }
-          if (!own) {
-            tc_commit(&a_empty[slot]);
-            ++a_cnt;
-          }
+          __syncwarp();
+          acc = 1;
+          if (!own) ++a_cnt;
         }
         if (!ok) break;
-        tc_commit(s_full);
+        if (elect_one()) tc_commit(s_full);
+        __syncwarp();
         ++b_cnt;
-        if (i > 0 && !(ok = issue_pv(prev_gs, prev_tg, i == 1))) break;
-        prev_gs = gs;
-        prev_tg = tg;
+        // The previous tile's P*V must be out before this tile's is queued.
+        if (!(ok = flush_pv())) break;
+        pv_pending = true;
+        pv_first = (i == 0);
+        pv_gs = gs;
+        pv_tg = tg;
+        pv_seg = seg_k;
         ++tg;
       }
-      if (ok && n > 0) ok = issue_pv(prev_gs, prev_tg, n == 1);
       ++seg_k;
     }
-    tc_commit(final_bar);
-    mbar_wait(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
+    if (ok) flush_pv();
+    if (elect_one()) tc_commit(final_bar);
+    __syncwarp();
+    mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
   } else if (warp >= 4) {
     // ------------------------------------------- softmax and epilogue (WG 1)
     const int r = tid - 128;
@@ -339,6 +415,10 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUt
           m_used = mt;
           resc = true;
         }
+        float psum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(exp2f(s[2 * u] - m_used), exp2f(s[2 * u + 1] - m_used), psum);
         if (i > 0) {
           if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
           tc_fence_after();
@@ -355,17 +435,11 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ CUt
           tmem_st_wait();
           l *= scale;
         }
-        float psum = 0.f;
         uint8_t* prow = sP + r * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint4 pk;
-          pk.x = pack_bf16(exp2f(s[8 * u + 0] - m_used), exp2f(s[8 * u + 1] - m_used), psum);
-          pk.y = pack_bf16(exp2f(s[8 * u + 2] - m_used), exp2f(s[8 * u + 3] - m_used), psum);
-          pk.z = pack_bf16(exp2f(s[8 * u + 4] - m_used), exp2f(s[8 * u + 5] - m_used), psum);
-          pk.w = pack_bf16(exp2f(s[8 * u + 6] - m_used), exp2f(s[8 * u + 7] - m_used), psum);
-          *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) = pk;
-        }
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         l += psum;
         if (valid < KT) {
           // Keys past the end: P is 0 there, but 0 * NaN would still poison O,

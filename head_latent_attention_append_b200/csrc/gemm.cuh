@@ -138,18 +138,37 @@ __device__ __forceinline__ void gemm_finish(const GemmArgs& a, int bz, int tile,
   __syncthreads();
   if (!is_last) return;
   __threadfence();
+  // The last split sums all splits in split order.  Each thread owns whole
+  // float4 groups of the tile and keeps eight loads in flight per group.
+  for (int q = threadIdx.x; q < BM * BN / 4; q += blockDim.x) {
+    const int r = q / (BN / 4), c = (q % (BN / 4)) * 4;
+    const float4* src = reinterpret_cast<const float4*>(base + r * BN + c);
+    float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 8 <= a.splits; s += 8) {
+      float4 v[8];
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    int r, c;
-    map(p, r, c);
-    float s0 = 0.f, s1 = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
-      float2 v = __ldcg(reinterpret_cast<const float2*>(base + (long long)s * (BM * BN) + r * BN + c));
-      s0 += v.x;
-      s1 += v.y;
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (long long)(s + u) * (BM * BN / 4));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc4.x += v[u].x;
+        acc4.y += v[u].y;
+        acc4.z += v[u].z;
+        acc4.w += v[u].w;
+      }
     }
-    int m = m0 + r, n = n0 + c;
-    if (m < a.M && n < a.N) epi(bz, m, n, s0, s1);
+    for (; s < a.splits; ++s) {
+      float4 v = __ldcg(src + (long long)s * (BM * BN / 4));
+      acc4.x += v.x;
+      acc4.y += v.y;
+      acc4.z += v.z;
+      acc4.w += v.w;
+    }
+    const int m = m0 + r, n = n0 + c;
+    if (m < a.M) {
+      if (n < a.N) epi(bz, m, n, acc4.x, acc4.y);
+      if (n + 2 < a.N) epi(bz, m, n + 2, acc4.z, acc4.w);
+    }
   }
   if (threadIdx.x == 0) *ctr = 0;
 }
@@ -181,7 +200,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const unsigned (&a)[4], 
 }
 
 template <class Epi>
-__global__ void __launch_bounds__(THREADS) kernel(GemmArgs a, Epi epi) {
+__global__ void __launch_bounds__(THREADS) gemm_bf16_kernel(GemmArgs a, Epi epi) {
   __shared__ __align__(128) __nv_bfloat16 As[STAGES][BM][PITCH];
   __shared__ __align__(128) __nv_bfloat16 Bs[STAGES][BN][PITCH];
   const int bz = blockIdx.z / a.splits, split = blockIdx.z % a.splits;
@@ -282,7 +301,7 @@ namespace gemm_f32 {
 constexpr int BM = 64, BN = 64, BK = 16, THREADS = 256;
 
 template <class Epi>
-__global__ void __launch_bounds__(THREADS) kernel(GemmArgs a, Epi epi) {
+__global__ void __launch_bounds__(THREADS) gemm_f32_kernel(GemmArgs a, Epi epi) {
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
   const int bz = blockIdx.z / a.splits, split = blockIdx.z % a.splits;

@@ -187,7 +187,7 @@ cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long
   a.M = M; a.N = N; a.K = K; a.batch = batch;
   const int tm = ceil_div(M, 64), tn = ceil_div(N, 64), tiles = tm * tn * batch;
   int splits = 1;
-  const int want = 2 * num_sms();
+  const int want = num_sms();
   if (tiles < want && tiles <= kCounterCap) {
     splits = ceil_div(want, tiles);
     splits = std::min(splits, std::max(1, K / 256));
@@ -202,8 +202,8 @@ cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long
   a.counters = at<int>(ws, P.counters);
   dim3 grid(tn, tm, batch * splits);
   ++g_launches;
-  if constexpr (sizeof(T) == 2) gemm_bf16::kernel<Epi><<<grid, gemm_bf16::THREADS, 0, st>>>(a, epi);
-  else gemm_f32::kernel<Epi><<<grid, gemm_f32::THREADS, 0, st>>>(a, epi);
+  if constexpr (sizeof(T) == 2) gemm_bf16::gemm_bf16_kernel<Epi><<<grid, gemm_bf16::THREADS, 0, st>>>(a, epi);
+  else gemm_f32::gemm_f32_kernel<Epi><<<grid, gemm_f32::THREADS, 0, st>>>(a, epi);
   return cudaGetLastError();
 }
 
@@ -311,17 +311,17 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     CUtensorMap map;
     if (!encode_cache_map(&map, cache, d_cr, (long long)num_pages * d.page_size)) return MLA_ERR_CUDA;
     attn_tc::Params pp{aa, ceil_div(d_cr, 64), d.d_c / 2};
-    if ((e = cudaFuncSetAttribute(attn_tc::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)attn_tc::SMEM_BYTES)))
       return cuda_status(e);
     ++g_launches;
     prof_mark(st, true);
-    attn_tc::kernel<<<dim3(W, 2), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
+    attn_tc::attn_tc_kernel<<<dim3(W, 2), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
   } else {
     size_t sm = attn_simt::smem_bytes(HG, d_cr);
-    auto kfn = attn_simt::kernel<T>;
+    auto kfn = attn_simt::attn_simt_kernel<T>;
     if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
       return cuda_status(e);
     ++g_launches;

@@ -21,6 +21,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// True on exactly one lane of a converged warp.  tcgen05 and TMA issue is
+// placed under it while the whole warp runs the same (uniform) control flow,
+// so the operands stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------- mbarriers
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -64,6 +73,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// Warp-uniform versions: every lane takes the same result.
+__device__ __forceinline__ bool mbar_try_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __shfl_sync(0xffffffffu, (int)mbar_try_wait(bar, parity), 0) != 0;
+}
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                               uint64_t limit_ns = 2000000000ull, bool honor_abort = true) {
+  bool ok = mbar_wait(bar, parity, abort, err, limit_ns, honor_abort);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ------------------------------------------------------------------- TMA
