@@ -1,37 +1,44 @@
-// Absorbed latent attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// Absorbed latent attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA),
+// one 2-CTA cluster per worker.
 //
 // What it computes is the same as attn_simt.cuh ("ai-decoupled-rope-mla",
 // absorbed score and output equations): for one query token, all of its heads
 // form the M = 128 rows (heads beyond n_h are zero rows), and for each 64-key
 // cache page
 //   S  = Q_abs [128 x d_cr] * page^T [d_cr x 64]      (content + position
-//        score in one contraction, because the cache row is [c | k_R] and the
-//        query row is [q~ | q_R], both pre-scaled by s*log2(e))
+//        score in one contraction: the cache row is [c | k_R] and the query
+//        row is [q~ | q_R], both pre-scaled by s*log2(e))
 //   P  = exp2(S - m)  (online softmax, running max m, running sum l)
-//   O += P [128 x 64] * page[:, latent half] [64 x d_c/2]
-// Only the cache tile is streamed; both products are dense because every
-// head shares the cache ("Latent Attention Meets RoPE": one shared position
-// key; the latent is shared by construction).
+//   O += P [128 x 64] * page[:, latent] [64 x d_c]
+// Both products are dense because every head shares the cache ("Latent
+// Attention Meets RoPE": one shared position key; the latent is shared by
+// construction).
 //
-// Layout decisions (B200): TMEM holds 512 columns x 128 lanes of fp32.  The
-// full latent accumulator of 128 heads x 512 would fill it, so each CTA of a
-// pair owns half of the latent output columns (blockIdx.y) and computes the
-// full score tile itself.  TMEM columns: O half [0, d_c/2), S [256, 320),
-// the first six 64-column chunks of Q [320, 512) (bf16 pairs packed in 32-bit
-// columns, the A operand of the score MMA); the remaining Q chunks are in
-// shared memory.  The cache is streamed by TMA in 64-key x 64-column chunks
-// (8 KB, 128-byte swizzle) through two rings: chunks only the score needs
-// (the other half of the latent and the RoPE key) are released as soon as
-// the score MMA has read them; the chunks of this CTA's own half stay until
-// the P*V MMA is done.  The two CTAs of a pair read the same pages at about
-// the same time, so the second read is served by L2.
+// B200 layout.  TMEM (128 lanes x 512 fp32 columns per SM) cannot hold the
+// 128 x 512 fp32 latent accumulator of one token next to anything else, so
+// the two CTAs of a cluster split the columns of the cache row:
+//   rank 0: latent columns [0, d_c/2)
+//   rank 1: latent columns [d_c/2, d_c) and the RoPE key columns.
+// Each CTA streams only its own columns of every page (no byte is read twice),
+// computes the partial score over them (all of its Q slice is the TMEM A
+// operand), and sends the partial, rounded to fp16, to its peer through
+// distributed shared memory.  Both CTAs add the two fp16 partials in fp32 --
+// the same two numbers, so both see bit-identical scores and run identical
+// softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
+// half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
+// P [480, 512).  Shared memory: a 4-deep ring of per-page column groups
+// (<= 5 chunks of 64 keys x 64 columns, 128-byte swizzle, loaded by TMA) and
+// two 16 KB exchange buffers, filled by the peer with asynchronous remote
+// stores that complete on this CTA's mbarrier.
 //
-// Warp roles (256 threads): warps 0 and 3 = TMA producers (one per ring),
-// warp 1 = MMA issuer (each runs warp-uniformly; one elected lane issues),
-// warp 2 = TMEM allocator,
-// warps 4-7 = softmax / epilogue (thread r owns row r = TMEM lane r).  Every
-// wait is bounded (sm100::mbar_wait).
+// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (both
+// warp-uniform; one elected lane issues), warp 2 = TMEM allocator, warps 4-11 =
+// two softmax / exchange / epilogue warpgroups (each owns half of the keys of
+// every row; thread r owns row r = TMEM lane r).  Every wait is bounded
+// (sm100::mbar_wait).
 #pragma once
+#include <cuda_fp16.h>
+
 #include "attn_simt.cuh"
 #include "sm100.cuh"
 
@@ -39,24 +46,21 @@ namespace mla {
 namespace attn_tc {
 using namespace sm100;
 
-constexpr int THREADS = 256;
-constexpr int KT = 64;                       // keys per tile (one page)
-constexpr int CHUNK_BYTES = 64 * 64 * 2;     // 64 keys x 64 bf16 columns
-constexpr int A_SLOTS = 8;
-constexpr int B_GROUPS = 3;
-constexpr int B_GROUP_BYTES = 4 * CHUNK_BYTES;
-constexpr int Q_TMEM_CHUNKS = 6;
-constexpr int Q_SMEM_CHUNKS = 3;
-constexpr int Q_CHUNK_BYTES = 128 * 128;
-constexpr int P_BYTES = 128 * 128;
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_COLS = 512;
+constexpr int THREADS = 384;
+constexpr int KT = 64;                        // keys per tile (one page)
+constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
+constexpr int MAX_OWN = 5;                    // chunks per CTA per page
+constexpr int GROUPS = 4;
+constexpr int GROUP_BYTES = MAX_OWN * CHUNK_BYTES;
+constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
 
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + A_SLOTS * CHUNK_BYTES;
-constexpr int OFF_Q = OFF_B + B_GROUPS * B_GROUP_BYTES;
-constexpr int OFF_P = OFF_Q + Q_SMEM_CHUNKS * Q_CHUNK_BYTES;
-constexpr int OFF_BAR = OFF_P + P_BYTES;
-constexpr int NUM_BARS = 2 * A_SLOTS + 2 * B_GROUPS + 7;
+constexpr int OFF_G = 0;
+constexpr int OFF_X = OFF_G + GROUPS * GROUP_BYTES;
+constexpr int OFF_MH = OFF_X + 2 * X_BYTES;       // half-row maxima [2][2][128] fp32
+constexpr int OFF_LS = OFF_MH + 2 * 2 * 128 * 4;  // half-row sums [2][128] fp32
+constexpr int OFF_BAR = OFF_LS + 2 * 128 * 4;
+constexpr int NUM_BARS = 2 * GROUPS + 2 + 7 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to 1024
@@ -64,8 +68,16 @@ constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to
 struct Params {
   AttnArgs a;
   int nkc;  // 64-column chunks per cache row (ceil(d_cr / 64))
-  int dh;   // latent columns per CTA (d_c / 2)
+  int npv;  // latent chunks per CTA (d_c / 128)
 };
+
+// 2^x with the MUFU ex2 instruction (flush-to-zero; ~2 ulp), used for the
+// softmax weights, which are rounded to bf16 right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b, float& sum) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -73,48 +85,82 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b, float& sum) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+// ------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Asynchronous 16-byte store into a peer CTA's shared memory; its bytes count
+// toward the transaction count of the peer's mbarrier `bar_cluster_addr`.
+__device__ __forceinline__ void st_async_peer_v4(uint32_t addr, uint4 v, uint32_t bar_cluster_addr) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_half2(uint32_t u) {
+  __half2 h = *reinterpret_cast<__half2*>(&u);
+  return __half22float2(h);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* a_full = bars;
-  uint64_t* a_empty = bars + A_SLOTS;
-  uint64_t* b_full = bars + 2 * A_SLOTS;
-  uint64_t* b_empty = b_full + B_GROUPS;
-  uint64_t* s_full = b_empty + B_GROUPS;
+  uint64_t* g_full = bars;
+  uint64_t* g_empty = bars + GROUPS;
+  uint64_t* x_full = bars + 2 * GROUPS;  // [2]
+  uint64_t* s_full = x_full + 2;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_full + 2;
   uint64_t* pv_done = s_full + 3;
   uint64_t* q_ready = s_full + 4;
   uint64_t* o_free = s_full + 5;
   uint64_t* final_bar = s_full + 6;
+  uint64_t* pair_bars = s_full + 7;  // [4]: the two softmax warps of a lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int w = blockIdx.x, half = blockIdx.y;
+  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+  const int w = blockIdx.x >> 1;
   const AttnArgs& a = p.a;
-  const int nkc = p.nkc, dh = p.dh, npv = dh / 64;
-  const int own0 = half * npv;  // first chunk of this CTA's latent half
+  const int nkc = p.nkc, npv = p.npv, dh = npv * 64;
+  const int c_lo = rank ? npv : 0;                 // first chunk this CTA loads
+  const int n_own = rank ? nkc - npv : npv;        // chunks this CTA loads per page
   const Seg* segs = a.sched.segs;
   const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
   if (tid == 32) {
-    for (int i = 0; i < A_SLOTS; ++i) {
-      mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 1);
+    for (int i = 0; i < GROUPS; ++i) {
+      mbar_init(&g_full[i], 1);
+      mbar_init(&g_empty[i], 1);
     }
-    for (int i = 0; i < B_GROUPS; ++i) {
-      mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
-    }
+    mbar_init(&x_full[0], 1);  // the receiver's expect_tx arrival + the peer's bytes
+    mbar_init(&x_full[1], 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_ready, 128);
+    mbar_init(s_free, 256);
+    mbar_init(p_ready, 256);
     mbar_init(pv_done, 1);
-    mbar_init(q_ready, 128);
-    mbar_init(o_free, 128);
+    mbar_init(q_ready, 256);
+    mbar_init(o_free, 256);
     mbar_init(final_bar, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -125,190 +171,91 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
   }
   if (tid == 0) tma_prefetch_desc(&tmap);
   __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 0 || warp == 3) {
-    // ----------------------------------------------------- TMA producers
-    // Warp 0 feeds the score-only ring, warp 3 the own-half ring; each walks
-    // every tile of the worker on its own, so neither ring waits for the
-    // other's slots.  The warp runs uniformly; one elected lane issues.
-    const bool ring_b = (warp == 3);
-    uint32_t cnt = 0;  // chunks (score-only ring) or tile groups (own-half ring) issued
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    uint32_t cnt = 0;
     bool ok = true;
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const Seg g = segs[si];
       const int seq = g.rb / a.n_q;
-      for (int t = g.t_lo; t < g.t_hi && ok; ++t) {
+      for (int t = g.t_lo; t < g.t_hi; ++t) {
         int page = a.page_table[(long long)seq * a.max_pages + t];
         if (page < 0 || page >= a.num_pages) {
-          if (!ring_b && elect_one()) flag_error(a.err, kErrBounds);
+          if (rank == 0 && elect_one()) flag_error(a.err, kErrBounds);
           page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
         }
-        const int y = page * KT;
-        if (ring_b) {
-          const uint32_t gs = cnt % B_GROUPS;
-          if (!(ok = mbar_wait_warp(&b_empty[gs], ((cnt / B_GROUPS) & 1) ^ 1, abort_flag, a.err))) break;
-          if (elect_one()) {
-            mbar_arrive_expect_tx(&b_full[gs], npv * CHUNK_BYTES);
-            for (int q = 0; q < npv; ++q)
-              tma_load_2d(smem + OFF_B + gs * B_GROUP_BYTES + q * CHUNK_BYTES, &tmap, (own0 + q) * 64, y,
-                          &b_full[gs]);
-          }
-          __syncwarp();
-          ++cnt;
-        } else {
-          for (int c = 0; c < nkc; ++c) {
-            if (c >= own0 && c < own0 + npv) continue;
-            const uint32_t slot = cnt % A_SLOTS;
-            if (!(ok = mbar_wait_warp(&a_empty[slot], ((cnt / A_SLOTS) & 1) ^ 1, abort_flag, a.err))) break;
-            if (elect_one()) {
-              mbar_arrive_expect_tx(&a_full[slot], CHUNK_BYTES);
-              tma_load_2d(smem + OFF_A + slot * CHUNK_BYTES, &tmap, c * 64, y, &a_full[slot]);
-            }
-            __syncwarp();
-            ++cnt;
-          }
+        const uint32_t gs = cnt % GROUPS;
+        if (!(ok = mbar_wait_warp(&g_empty[gs], ((cnt / GROUPS) & 1) ^ 1, abort_flag, a.err))) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&g_full[gs], n_own * CHUNK_BYTES);
+          for (int q = 0; q < n_own; ++q)
+            tma_load_2d(smem + OFF_G + gs * GROUP_BYTES + q * CHUNK_BYTES, &tmap, (c_lo + q) * 64, page * KT,
+                        &g_full[gs]);
         }
+        __syncwarp();
+        ++cnt;
       }
     }
     if (*abort_flag) {
       // Let every copy already issued land before the CTA can exit.
-      const uint32_t n = ring_b ? B_GROUPS : A_SLOTS;
-      uint64_t* full = ring_b ? b_full : a_full;
-      for (uint32_t q = 0; q < n && q < cnt; ++q) {
-        const uint32_t last = q + n * ((cnt - 1 - q) / n);
-        mbar_wait_warp(&full[q], (last / n) & 1, abort_flag, nullptr, 50000000ull, false);
+      for (uint32_t q = 0; q < GROUPS && q < cnt; ++q) {
+        const uint32_t last = q + GROUPS * ((cnt - 1 - q) / GROUPS);
+        mbar_wait_warp(&g_full[q], (last / GROUPS) & 1, abort_flag, nullptr, 50000000ull, false);
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    // Issue order per tile: the score MMA of tile t (own-half chunks first,
-    // they were prefetched furthest ahead), and the P*V MMA of tile t-1 as
-    // soon as its P is ready -- polled while waiting for score data, so a
-    // late chunk never holds back the release of the own-half ring.  The
-    // whole warp runs this loop with uniform values; one elected lane issues
-    // each tcgen05 instruction.
+    // Per tile: the partial score MMA of tile t, then the P*V MMA of tile t-1.
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);
     const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
-    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q;
-    const uint32_t sA = smem_u32(smem + OFF_A), sB = smem_u32(smem + OFF_B);
-    const uint32_t sQ = smem_u32(smem + OFF_Q), sP = smem_u32(smem + OFF_P);
-    uint32_t a_cnt = 0, b_cnt = 0, tg = 0, seg_k = 0;
+    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q, tP = tbase + TM_P;
+    const uint32_t sG = smem_u32(smem + OFF_G);
+    uint32_t tg = 0, seg_k = 0;
     bool ok = true;
-    bool pv_pending = false, pv_first = false;
-    uint32_t pv_gs = 0, pv_tg = 0, pv_seg = 0;
-    // Issues the pending P*V MMA if its inputs are ready; never blocks.
-    auto try_pv = [&]() {
-      if (!pv_pending || !mbar_try_wait_warp(p_ready, pv_tg & 1)) return;
-      if (pv_first && pv_seg > 0 && !mbar_try_wait_warp(o_free, (pv_seg - 1) & 1)) return;
+    // P*V of the previous tile, issued right after the next score MMA.
+    auto issue_pv = [&](uint32_t gs, uint32_t tile_tg, bool first, uint32_t seg) -> bool {
+      if (!mbar_wait_warp(p_ready, tile_tg & 1, abort_flag, a.err)) return false;
+      if (first && seg > 0 && !mbar_wait_warp(o_free, (seg - 1) & 1, abort_flag, a.err)) return false;
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sP + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sB + pv_gs * B_GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024);
-          mma_ss(tO, ad, bd, idPV, (pv_first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < KT / 16; ++kk)
+          mma_ts(tO, tP + kk * 8, sdesc_sw128(sG + gs * GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
+                 (first && kk == 0) ? 0u : 1u);
         tc_commit(pv_done);
-        tc_commit(&b_empty[pv_gs]);
+        tc_commit(&g_empty[gs]);
       }
       __syncwarp();
-      pv_pending = false;
-    };
-    // Bounded wait on `bar` that keeps issuing the pending P*V meanwhile.
-    auto wait_polling = [&](uint64_t* bar, uint32_t parity) -> bool {
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait_warp(bar, parity)) {
-        try_pv();
-        int stop = 0;
-        if (*abort_flag) stop = 1;
-        else if (globaltimer_ns() - t0 > 2000000000ull) stop = 2;
-        stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (stop) {
-          if (stop == 2 && elect_one()) {
-            *abort_flag = 1;
-            flag_error(a.err, kErrTimeout);
-          }
-          __syncwarp();
-          return false;
-        }
-      }
       return true;
     };
-    auto flush_pv = [&]() -> bool {
-      const uint64_t t0 = globaltimer_ns();
-      while (pv_pending) {
-        try_pv();
-        if (!pv_pending) break;
-        int stop = 0;
-        if (*abort_flag) stop = 1;
-        else if (globaltimer_ns() - t0 > 2000000000ull) stop = 2;
-        stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (stop) {
-          if (stop == 2 && elect_one()) {
-            *abort_flag = 1;
-            flag_error(a.err, kErrTimeout);
-          }
-          __syncwarp();
-          return false;
-        }
-      }
-      return true;
-    };
+    bool pv_pending = false, pv_first = false;
+    uint32_t pv_gs = 0, pv_tg = 0, pv_seg = 0;
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
       const Seg g = segs[si];
       const int n = g.t_hi - g.t_lo;
-      if (!(ok = wait_polling(q_ready, seg_k & 1))) break;
+      if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
       tc_fence_after();
-      for (int i = 0; i < n && ok; ++i) {
-        if (tg > 0 && !(ok = wait_polling(s_free, (tg - 1) & 1))) break;
+      for (int i = 0; i < n; ++i) {
+        if (tg > 0 && !(ok = mbar_wait_warp(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
+        const uint32_t gs = tg % GROUPS;
+        if (!(ok = mbar_wait_warp(&g_full[gs], (tg / GROUPS) & 1, abort_flag, a.err))) break;
         tc_fence_after();
-        const uint32_t gs = b_cnt % B_GROUPS;
-        uint32_t acc = 0;
-        for (int k2 = 0; k2 < nkc; ++k2) {
-          // own-half chunks first, then the rest in column order
-          int c;
-          if (k2 < npv) c = own0 + k2;
-          else {
-            const int j = k2 - npv;
-            c = (j < own0) ? j : j + npv;
-          }
-          const bool own = k2 < npv;
-          uint32_t bsrc, slot = 0;
-          if (own) {
-            if (k2 == 0 && !(ok = wait_polling(&b_full[gs], (b_cnt / B_GROUPS) & 1))) break;
-            bsrc = sB + gs * B_GROUP_BYTES + k2 * CHUNK_BYTES;
-          } else {
-            slot = a_cnt % A_SLOTS;
-            if (!(ok = wait_polling(&a_full[slot], (a_cnt / A_SLOTS) & 1))) break;
-            bsrc = sA + slot * CHUNK_BYTES;
-          }
-          tc_fence_after();
-          if (elect_one()) {
-            if (c < Q_TMEM_CHUNKS) {
+        if (elect_one()) {
+          const uint32_t gb = sG + gs * GROUP_BYTES;
+          for (int q = 0; q < n_own; ++q) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_ts(tS, tQ + c * 32 + k * 8, sdesc_sw128(bsrc + k * 32, 16, 1024), idS, (acc | k) ? 1u : 0u);
-            } else {
-              const uint32_t qa = sQ + (c - Q_TMEM_CHUNKS) * Q_CHUNK_BYTES;
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_ss(tS, sdesc_sw128(qa + k * 32, 16, 1024), sdesc_sw128(bsrc + k * 32, 16, 1024), idS,
-                       (acc | k) ? 1u : 0u);
-            }
-            if (!own) tc_commit(&a_empty[slot]);
+            for (int k = 0; k < 4; ++k)
+              mma_ts(tS, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
+                     (q | k) ? 1u : 0u);
           }
-          __syncwarp();
-          acc = 1;
-          if (!own) ++a_cnt;
+          tc_commit(s_full);
         }
-        if (!ok) break;
-        if (elect_one()) tc_commit(s_full);
         __syncwarp();
-        ++b_cnt;
-        // The previous tile's P*V must be out before this tile's is queued.
-        if (!(ok = flush_pv())) break;
+        if (pv_pending && !(ok = issue_pv(pv_gs, pv_tg, pv_first, pv_seg))) break;
         pv_pending = true;
         pv_first = (i == 0);
         pv_gs = gs;
@@ -318,55 +265,65 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       }
       ++seg_k;
     }
-    if (ok) flush_pv();
+    if (ok && pv_pending) ok = issue_pv(pv_gs, pv_tg, pv_first, pv_seg);
     if (elect_one()) tc_commit(final_bar);
     __syncwarp();
     mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
   } else if (warp >= 4) {
-    // ------------------------------------------- softmax and epilogue (WG 1)
-    const int r = tid - 128;
+    // ------------------------------- softmax, score exchange and epilogue
+    // Two warpgroups: WG h (warps 4+4h .. 7+4h) owns keys [32h, 32h + 32) of
+    // every row; thread r of a WG owns row r (= TMEM lane r).  The two threads
+    // of a row meet at a 64-thread named barrier (their warps share a lane
+    // quarter) to agree on the row maximum.
+    const int h = warp >= 8 ? 1 : 0;
+    const int r = tid - 128 - 128 * h;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O, tQ = tbase + lane_off + TM_Q;
-    uint8_t* sP = smem + OFF_P;
-    uint8_t* sQ = smem + OFF_Q;
-    uint8_t* sB = smem + OFF_B;
+    const uint32_t tS = tbase + lane_off + TM_S + 32 * h, tO = tbase + lane_off + TM_O;
+    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P + 16 * h;
+    uint64_t* pair_bar = &pair_bars[warp & 3];
+    uint32_t pair_phase = 0;
+    uint8_t* sG = smem + OFF_G;
+    uint8_t* sX = smem + OFF_X;
+    float* mh = reinterpret_cast<float*>(smem + OFF_MH);
+    float* ls = reinterpret_cast<float*>(smem + OFF_LS);
+    const uint32_t peer_x = map_peer(smem_u32(sX), peer);
+    const uint32_t peer_xbar0 = map_peer(smem_u32(&x_full[0]), peer);
+    const uint32_t peer_xbar1 = map_peer(smem_u32(&x_full[1]), peer);
     const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
-    const int nq_tmem = min(nkc, Q_TMEM_CHUNKS);
-    uint32_t tg = 0, b_cnt = 0;
+    const int hc0 = h * (dh / 64), hc1 = hc0 + dh / 64;  // this WG's 32-column chunks of O
+    uint32_t tg = 0;
     bool ok = true;
 
+    // Meeting point of the two threads of a row (bounded, like every wait).
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(pair_bar);
+      bool r_ok = mbar_wait(pair_bar, pair_phase & 1, abort_flag, a.err);
+      ++pair_phase;
+      return __all_sync(0xffffffffu, r_ok);
+    };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
       return __all_sync(0xffffffffu, r_ok);
     };
-    // Q row r of token rb into TMEM (chunks < 6) and swizzled smem (the rest).
+    // Row r of this CTA's Q slice (chunks c_lo .. c_lo + n_own - 1) into TMEM;
+    // the two warpgroups take alternate chunks.
     auto load_q = [&](int rb) {
       const uint4* src =
           (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
-      for (int c = 0; c < nq_tmem; ++c) {
+      for (int q = h; q < n_own; q += 2) {
         uint32_t wv[32];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int col = c * 64 + u * 8;
+          const int col = (c_lo + q) * 64 + u * 8;
           uint4 v = (src && col < a.d_cr) ? __ldg(src + col / 8) : make_uint4(0, 0, 0, 0);
           wv[4 * u + 0] = v.x;
           wv[4 * u + 1] = v.y;
           wv[4 * u + 2] = v.z;
           wv[4 * u + 3] = v.w;
         }
-        tmem_st32(tQ + c * 32, wv);
+        tmem_st32(tQ + q * 32, wv);
       }
       tmem_st_wait();
-      for (int c = nq_tmem; c < nkc; ++c) {
-        uint8_t* chunk = sQ + (c - Q_TMEM_CHUNKS) * Q_CHUNK_BYTES + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int col = c * 64 + u * 8;
-          uint4 v = (src && col < a.d_cr) ? __ldg(src + col / 8) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(chunk + ((u ^ (r & 7)) << 4)) = v;
-        }
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(q_ready);
     };
@@ -380,29 +337,68 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       float m_used = -INFINITY, l = 0.f;
       for (int i = 0; i < n; ++i) {
         const int t = g.t_lo + i;
+        const uint32_t xb = tg & 1;
         if (!(ok = wait_all(s_full, tg & 1))) break;
         tc_fence_after();
-        float s[64];
+        // Own partial score (this WG's 32 keys), rounded to fp16; the same
+        // values go to the peer.
+        uint32_t own[16];
         {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tS, v0);
-          tmem_ld32(tS + 32, v1);
+          uint32_t v[32];
+          tmem_ld32(tS, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            s[j] = __uint_as_float(v0[j]);
-            s[32 + j] = __uint_as_float(v1[j]);
-          }
+          for (int j = 0; j < 16; ++j) own[j] = pack_half2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
         }
         tc_fence_before();
         mbar_arrive(s_free);
-        const int valid = min(KT, nkeys - t * KT);
-        float mt = -INFINITY;
+        {
+          const uint32_t dst = peer_x + xb * X_BYTES + r * 128 + h * 64;
+          const uint32_t pbar = xb ? peer_xbar1 : peer_xbar0;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          if (j >= valid) s[j] = -INFINITY;
-          mt = fmaxf(mt, s[j]);
+          for (int u = 0; u < 4; ++u)
+            st_async_peer_v4(dst + u * 16, make_uint4(own[4 * u], own[4 * u + 1], own[4 * u + 2], own[4 * u + 3]),
+                             pbar);
         }
+        if (h == 0 && r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
+        if (!(ok = wait_all(&x_full[xb], (tg >> 1) & 1))) break;
+        float s[32];
+        {
+          const uint4* src = reinterpret_cast<const uint4*>(sX + xb * X_BYTES + r * 128 + h * 64);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 pv = src[u];
+            const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 mine = unpack_half2(own[4 * u + e]);
+              const float2 theirs = unpack_half2(pw[e]);
+              s[8 * u + 2 * e] = mine.x + theirs.x;
+              s[8 * u + 2 * e + 1] = mine.y + theirs.y;
+            }
+          }
+        }
+        const int valid = min(KT, nkeys - t * KT) - 32 * h;  // valid keys among this WG's 32
+        if (valid < 32) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j >= valid) s[j] = -INFINITY;
+        }
+        float mt;
+        {
+          float mx[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
+#pragma unroll
+          for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+          float* slot = mh + (tg & 1) * 256;
+          slot[h * 128 + r] = mx[0];
+          ok = pair_sync();
+          mt = fmaxf(slot[r], slot[128 + r]);
+        }
+        if (!ok) break;
         // Running max with lazy rescaling: O and l stay relative to m_used
         // until a tile's max exceeds it by more than 2^8.
         bool resc = false;
@@ -411,20 +407,31 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
           m_used = mt;
           l = 0.f;
         } else if (mt > m_used + 8.f) {
-          scale = exp2f(m_used - mt);
+          scale = fast_exp2(m_used - mt);
           m_used = mt;
           resc = true;
         }
-        float psum = 0.f;
-        uint32_t pk[32];
+        uint32_t pk[16];
+        float psum;
+        {
+          float ps[16];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(exp2f(s[2 * u] - m_used), exp2f(s[2 * u + 1] - m_used), psum);
+          for (int u = 0; u < 16; ++u) {
+            ps[u] = 0.f;
+            pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u]);
+          }
+#pragma unroll
+          for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
+          psum = ps[0];
+        }
         if (i > 0) {
           if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
           tc_fence_after();
         }
         if (__any_sync(0xffffffffu, resc)) {
-          for (int cc = 0; cc < dh / 32; ++cc) {
+          for (int cc = hc0; cc < hc1; ++cc) {
             uint32_t v[32];
             tmem_ld32(tO + cc * 32, v);
             tmem_ld_wait();
@@ -432,46 +439,47 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
             tmem_st32(tO + cc * 32, v);
           }
-          tmem_st_wait();
           l *= scale;
         }
-        uint8_t* prow = sP + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        tmem_st16(tP, pk);
+        tmem_st_wait();
         l += psum;
-        if (valid < KT) {
+        const int valid_all = min(KT, nkeys - t * KT);
+        if (valid_all < KT) {
           // Keys past the end: P is 0 there, but 0 * NaN would still poison O,
-          // so clear those rows of this tile's own-half chunks.
-          uint8_t* gb = sB + (b_cnt % B_GROUPS) * B_GROUP_BYTES;
-          const int rows = KT - valid, units = rows * 8 * npv;
-          for (int x = r; x < units; x += 128) {
+          // so clear those rows of this tile's latent chunks.
+          uint8_t* gb = sG + (tg % GROUPS) * GROUP_BYTES;
+          const int rows = KT - valid_all, units = rows * 8 * npv;
+          for (int x = r + 128 * h; x < units; x += 256) {
             const int q = x / (rows * 8), rem = x - q * rows * 8;
-            *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+            *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_ready);
         ++tg;
-        ++b_cnt;
       }
       if (!ok) break;
       if (si + 1 < seg_hi) load_q(segs[si + 1].rb);
       if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
       tc_fence_after();
+      // Row sum: both halves add the two partial sums in the same order.
+      ls[h * 128 + r] = l;
+      if (!(ok = pair_sync())) break;
+      const float lrow = ls[r] + ls[128 + r];
+      if (!(ok = pair_sync())) break;  // both have read before the next segment's write
       // Epilogue: a whole row block is normalised into obar (bf16); a piece of
       // a split row block leaves its unnormalised sum and (m, l) in its slot.
       const bool whole = g.slot < 0;
-      const float inv = 1.f / l;
-      for (int cc = 0; cc < dh / 32; ++cc) {
+      const float inv = 1.f / lrow;
+      for (int cc = hc0; cc < hc1; ++cc) {
         uint32_t v[32];
         tmem_ld32(tO + cc * 32, v);
         tmem_ld_wait();
         if (r < a.n_h) {
-          const int col = half * dh + cc * 32;
+          const int col = (int)rank * dh + cc * 32;
           if (whole) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.obar) +
                                                   ((long long)rb * a.n_h + r) * a.d_c + col);
@@ -492,9 +500,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
           }
         }
       }
-      if (!whole && half == 0 && r < a.n_h) {
+      if (!whole && rank == 0 && h == 0 && r < a.n_h) {
         a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 0] = m_used;
-        a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = l;
+        a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = lrow;
       }
       tc_fence_before();
       mbar_arrive(o_free);
@@ -503,6 +511,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still write into it
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tbase, TM_COLS);

@@ -310,13 +310,13 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   if constexpr (kTensorCores) {
     CUtensorMap map;
     if (!encode_cache_map(&map, cache, d_cr, (long long)num_pages * d.page_size)) return MLA_ERR_CUDA;
-    attn_tc::Params pp{aa, ceil_div(d_cr, 64), d.d_c / 2};
+    attn_tc::Params pp{aa, ceil_div(d_cr, 64), d.d_c / 128};
     if ((e = cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)attn_tc::SMEM_BYTES)))
       return cuda_status(e);
     ++g_launches;
     prof_mark(st, true);
-    attn_tc::attn_tc_kernel<<<dim3(W, 2), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
+    attn_tc::attn_tc_kernel<<<dim3(2 * W), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
   } else {
