@@ -170,13 +170,17 @@ inline size_t smem_bytes(int HG, int d_cr) {
 // ------------------------------------------------------------ combine -----
 // Merges the partial slots of each split row block (log-sum-exp in base 2):
 //   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  obar = sum_s 2^(m_s - m) O_s / l.
-// Slots are visited in segment order, so the result is deterministic.
+// Block = (split row block, 8 heads), one warp per head, lanes across the
+// latent columns.  Slots are visited in segment order, so the result is
+// deterministic.
 template <typename T>
-__global__ void combine_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
   const Sched& S = a.sched;
   const int idx = blockIdx.x;
   if (idx >= S.split_rbs[0]) return;
-  const int rb = S.split_rbs[1 + idx], h = blockIdx.y;
+  const int rb = S.split_rbs[1 + idx];
+  const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (h >= a.n_h) return;
   const int s0 = S.rb_seg_first[rb], s1 = S.rb_seg_first[rb + 1];
   float m = -INFINITY;
   for (int s = s0; s < s1; ++s) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
@@ -187,14 +191,23 @@ __global__ void combine_kernel(AttnArgs a) {
   }
   const float inv = 1.f / l;
   T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
-  for (int j = threadIdx.x; j < a.d_c; j += blockDim.x) {
-    float acc = 0.f;
+  for (int j0 = 0; j0 < a.d_c; j0 += 128) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int s = s0; s < s1; ++s) {
-      int slot = S.segs[s].slot;
-      float wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
-      acc += wgt * a.part_o[((long long)slot * a.n_h + h) * a.d_c + j];
+      const int slot = S.segs[s].slot;
+      const float wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
+      const float* src = a.part_o + ((long long)slot * a.n_h + h) * a.d_c + j0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = q * 32 + lane;
+        if (j0 + j < a.d_c) acc[q] += wgt * __ldcg(src + j);
+      }
     }
-    out[j] = from_f32<T>(acc * inv);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q * 32 + lane;
+      if (j < a.d_c) out[j] = from_f32<T>(acc[q] * inv);
+    }
   }
 }
 

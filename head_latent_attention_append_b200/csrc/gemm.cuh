@@ -4,11 +4,9 @@
 // is exactly y = W x applied to every token.  The epilogue functor receives
 // adjacent column pairs (n even) and places, rotates and rounds them.
 //
-// Two main loops share the split-K bookkeeping and the epilogue:
-//   * bf16: mma.sync m16n8k16 tensor-core tiles fed by a 3-stage cp.async
-//     pipeline (used for the weight-streaming projections);
-//   * fp32: FFMA tiles (the fp32 path must stay within 1e-4, which excludes
-//     single-pass TF32).
+// This file holds the epilogue functors shared with the tensor-core GEMM
+// (gemm_tc.cuh) and the fp32 CUDA-core main loop (the fp32 path must stay
+// within 1e-4, which excludes single-pass TF32).
 // Split-K: every split writes its fp32 tile to scratch and bumps a per-tile
 // counter; the last split to arrive sums all splits in split order (so the
 // result is deterministic) and runs the epilogue, then re-arms the counter.
@@ -172,129 +170,6 @@ __device__ __forceinline__ void gemm_finish(const GemmArgs& a, int bz, int tile,
   }
   if (threadIdx.x == 0) *ctr = 0;
 }
-
-// ------------------------------------------------------------ bf16 kernel
-namespace gemm_bf16 {
-constexpr int BM = 64, BN = 64, BK = 32, STAGES = 3, PITCH = BK + 8, THREADS = 128;
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int bytes) {
-  unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ __forceinline__ void ldmatrix_x4(unsigned (&r)[4], const void* p) {
-  unsigned s = (unsigned)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(s));
-}
-__device__ __forceinline__ void mma16816(float (&d)[4], const unsigned (&a)[4], unsigned b0, unsigned b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-template <class Epi>
-__global__ void __launch_bounds__(THREADS) gemm_bf16_kernel(GemmArgs a, Epi epi) {
-  __shared__ __align__(128) __nv_bfloat16 As[STAGES][BM][PITCH];
-  __shared__ __align__(128) __nv_bfloat16 Bs[STAGES][BN][PITCH];
-  const int bz = blockIdx.z / a.splits, split = blockIdx.z % a.splits;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-  const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A) + bz * a.strideA;
-  const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(a.B) + bz * a.strideB;
-  const int k_begin = split * a.kchunk;
-  const int k_end = min(a.K, k_begin + a.kchunk);
-  const int nk = k_end > k_begin ? ceil_div(k_end - k_begin, BK) : 0;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wm = warp >> 1, wn = warp & 1;
-
-  auto load = [&](int stage, int k0) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      int idx = tid + i * THREADS;  // 256 chunks of 16 B per operand tile
-      int r = idx >> 2, ck = (idx & 3) * 8;
-      int gk = k0 + ck;
-      {
-        int gm = m0 + r;
-        bool ok = gm < a.M && gk < k_end;
-        const void* src = ok ? (const void*)(A + (long long)gm * a.lda + gk) : (const void*)A;
-        cp_async16(&As[stage][r][ck], src, ok ? 16 : 0);
-      }
-      {
-        int gn = n0 + r;
-        bool ok = gn < a.N && gk < k_end;
-        const void* src = ok ? (const void*)(B + (long long)gn * a.ldb + gk) : (const void*)B;
-        cp_async16(&Bs[stage][r][ck], src, ok ? 16 : 0);
-      }
-    }
-  };
-
-  float acc[2][4][4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < nk) load(s, k_begin + s * BK);
-    cp_async_commit();
-  }
-  for (int kt = 0; kt < nk; ++kt) {
-    cp_async_wait<STAGES - 2>();
-    __syncthreads();
-    int nxt = kt + STAGES - 1;
-    if (nxt < nk) load(nxt % STAGES, k_begin + nxt * BK);
-    cp_async_commit();
-    const int st = kt % STAGES;
-#pragma unroll
-    for (int kk = 0; kk < BK; kk += 16) {
-      unsigned af[2][4], bfr[2][4];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-        ldmatrix_x4(af[i], &As[st][wm * 32 + i * 16 + (lane & 15)][kk + (lane >> 4) * 8]);
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-        ldmatrix_x4(bfr[j], &Bs[st][wn * 32 + j * 16 + (lane & 7) + (lane >> 4) * 8][kk + ((lane >> 3) & 1) * 8]);
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          mma16816(acc[i][2 * j], af[i], bfr[j][0], bfr[j][1]);
-          mma16816(acc[i][2 * j + 1], af[i], bfr[j][2], bfr[j][3]);
-        }
-    }
-  }
-  cp_async_wait<0>();
-
-  // Pair p = (i, j, half): rows wm*32 + i*16 + g (+8), cols wn*32 + j*8 + 2t.
-  float pairs[16][2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        pairs[(i * 4 + j) * 2 + h][0] = acc[i][j][2 * h];
-        pairs[(i * 4 + j) * 2 + h][1] = acc[i][j][2 * h + 1];
-      }
-  const int g = lane >> 2, t4 = lane & 3;
-  auto map = [&](int p, int& r, int& c) {
-    int h = p & 1, j = (p >> 1) & 3, i = p >> 3;
-    r = wm * 32 + i * 16 + g + h * 8;
-    c = wn * 32 + j * 8 + 2 * t4;
-  };
-  gemm_finish<BM, BN, 16>(a, bz, tile, split, m0, n0, pairs, map, epi);
-}
-}  // namespace gemm_bf16
 
 // ------------------------------------------------------------ fp32 kernel
 namespace gemm_f32 {

@@ -16,6 +16,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_tc.cuh"
 #include "prep.cuh"
 #include "sched.cuh"
 
@@ -59,9 +60,46 @@ constexpr double kLog2e = 1.4426950408889634074;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  static thread_local int cached_dev = -1, cached_n = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cached_n;
+  if (dev != cached_dev) {
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached_n = n > 0 ? n : 148;
+    cached_dev = dev;
+  }
+  return cached_n;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), so
+// later calls, including ones made during CUDA graph capture, skip it.
+template <class F>
+cudaError_t set_smem_once(F* fn, size_t bytes) {
+  struct Entry {
+    const void* fn;
+    unsigned long long devices;
+  };
+  static std::mutex mu;
+  static Entry table[64];
+  static int used = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* ent = nullptr;
+  for (int i = 0; i < used; ++i)
+    if (table[i].fn == reinterpret_cast<const void*>(fn)) ent = &table[i];
+  if (ent && (ent->devices & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (!ent && used < 64) ent = &table[used++];
+  if (ent) {
+    ent->fn = reinterpret_cast<const void*>(fn);
+    ent->devices |= bit;
+  }
+  return cudaSuccess;
 }
 
 mla_status check_dims(const mla_dims* d) {
@@ -175,12 +213,100 @@ bool encode_cache_map(CUtensorMap* map, const void* cache, int d_cr, long long r
   return r == CUDA_SUCCESS;
 }
 
+// bf16 tensor maps with 128-byte swizzle for the projection GEMMs.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, long long dim0, long long dim1, long long stride1_elems,
+                    int box0, int box1) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)dim0, (cuuint64_t)dim1};
+  cuuint64_t gstride[1] = {(cuuint64_t)stride1_elems * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box0, (cuuint32_t)box1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool encode_bf16_3d(CUtensorMap* map, const void* base, long long dim0, long long dim1, long long dim2,
+                    long long stride1_elems, long long stride2_elems, int box0, int box1, int box2) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
+  cuuint64_t gstride[2] = {(cuuint64_t)stride1_elems * 2, (cuuint64_t)stride2_elems * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, (cuuint32_t)box2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// tcgen05 projection GEMM: C[b][m][n] = sum_k A[b][m][k] * B[b][n][k] with A
+// the activations (m = token) and B the weights (n = output column); the
+// kernel runs it as D = W X^T (weights as the MMA's M).  `partial_floats`
+// bounds the split-K scratch.
+template <int BN, class Epi>
+cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
+                           int M, int N, int K, int batch, const Epi& epi, float* partial, long long partial_floats,
+                           cudaStream_t st) {
+  CUtensorMap mapW, mapX;
+  // Weights: batches are contiguous row blocks of N rows.
+  if (batch > 1 && sB != (long long)N * ldb) return cudaErrorInvalidValue;
+  if (!encode_bf16_2d(&mapW, B, K, (long long)batch * N, ldb, gemm_tc::BK, gemm_tc::BM)) return cudaErrorInvalidValue;
+  const bool x3d = batch > 1;
+  if (x3d) {
+    if (!encode_bf16_3d(&mapX, A, K, batch, M, sA, lda, gemm_tc::BK, 1, BN)) return cudaErrorInvalidValue;
+  } else if (!encode_bf16_2d(&mapX, A, K, M, lda, gemm_tc::BK, BN)) {
+    return cudaErrorInvalidValue;
+  }
+  const int tm = ceil_div(N, gemm_tc::BM), tn = ceil_div(M, BN), tiles = tm * tn * batch;
+  const int nk = ceil_div(K, gemm_tc::BK);
+  int splits = 1;
+  const int sms = num_sms();
+  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), ceil_div(sms, tiles));
+  while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
+  const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
+  splits = ceil_div(K, kchunk);
+  gemm_tc::Args g{N, M, K, splits, kchunk, N, x3d ? 1 : 0, partial};
+  const size_t smem = gemm_tc::smem_bytes<BN>();
+  auto kfn = gemm_tc::gemm_tc_kernel<BN, Epi>;
+  cudaError_t e = set_smem_once(kfn, smem);
+  if (e != cudaSuccess) return e;
+  ++g_launches;
+  kfn<<<dim3(tm, tn, batch * splits), gemm_tc::THREADS, smem, st>>>(mapW, mapX, g, epi);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (splits > 1) {
+    ++g_launches;
+    gemm_tc::splitk_reduce_kernel<BN, Epi><<<dim3(tm, tn * (BN / 8), batch), 256, 0, st>>>(g, epi);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
 // ----------------------------------------------------------- GEMM launcher
+template <class Epi>
+cudaError_t gemm_simt(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB, int M,
+                      int N, int K, int batch, const Epi& epi, void* ws, const Plan& P, cudaStream_t st,
+                      int tile_split_cap);
+
 template <typename T, class Epi>
 cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                  int M, int N, int K, int batch, const Epi& epi, void* ws, const Plan& P,
                  cudaStream_t st, int tile_split_cap = kSplitKTileSplits) {
   if (M <= 0 || N <= 0) return cudaSuccess;
+  if constexpr (sizeof(T) == 2) {
+    const long long cap = (long long)tile_split_cap * 64 * 64;
+    if (M <= 512)
+      return gemm_tc_launch<64>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st);
+    return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st);
+  } else {
+    return gemm_simt(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, ws, P, st, tile_split_cap);
+  }
+}
+
+// fp32 CUDA-core GEMM (the fp32 path).
+template <class Epi>
+cudaError_t gemm_simt(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB, int M,
+                      int N, int K, int batch, const Epi& epi, void* ws, const Plan& P, cudaStream_t st,
+                      int tile_split_cap) {
   GemmArgs a{};
   a.A = A; a.lda = lda; a.strideA = sA;
   a.B = B; a.ldb = ldb; a.strideB = sB;
@@ -202,8 +328,7 @@ cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long
   a.counters = at<int>(ws, P.counters);
   dim3 grid(tn, tm, batch * splits);
   ++g_launches;
-  if constexpr (sizeof(T) == 2) gemm_bf16::gemm_bf16_kernel<Epi><<<grid, gemm_bf16::THREADS, 0, st>>>(a, epi);
-  else gemm_f32::gemm_f32_kernel<Epi><<<grid, gemm_f32::THREADS, 0, st>>>(a, epi);
+  gemm_f32::gemm_f32_kernel<Epi><<<grid, gemm_f32::THREADS, 0, st>>>(a, epi);
   return cudaGetLastError();
 }
 
@@ -311,9 +436,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     CUtensorMap map;
     if (!encode_cache_map(&map, cache, d_cr, (long long)num_pages * d.page_size)) return MLA_ERR_CUDA;
     attn_tc::Params pp{aa, ceil_div(d_cr, 64), d.d_c / 128};
-    if ((e = cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)attn_tc::SMEM_BYTES)))
-      return cuda_status(e);
+    if ((e = set_smem_once(attn_tc::attn_tc_kernel, attn_tc::SMEM_BYTES))) return cuda_status(e);
     ++g_launches;
     prof_mark(st, true);
     attn_tc::attn_tc_kernel<<<dim3(2 * W), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, pp);
@@ -323,7 +446,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     size_t sm = attn_simt::smem_bytes(HG, d_cr);
     auto kfn = attn_simt::attn_simt_kernel<T>;
     if ((e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
-      return cuda_status(e);
+      return cuda_status(e);  // fp32 path: size depends on the head group
     ++g_launches;
     prof_mark(st, true);
     kfn<<<dim3(W, G), attn_simt::THREADS, sm, st>>>(aa, HG);
@@ -332,7 +455,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   }
   {
     ++g_launches;
-    combine_kernel<T><<<dim3(2 * W, d.n_h), 128, 0, st>>>(aa);
+    combine_kernel<T><<<dim3(2 * W, ceil_div(d.n_h, 8)), 256, 0, st>>>(aa);
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (7) o_h = W_UV,h obar_h.
