@@ -92,14 +92,22 @@ def dist_setup():
     return ws, rank, local
 
 
-def max_over_ranks(x: float, ws: int) -> float:
+def max_over_ranks(x: float, ws: int, device: str = "cuda") -> float:
+    """Largest value of x over all ranks (x is each rank's device time)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(bytes_per_rank: int, ms_local: float, ws: int, device: str = "cuda"):
+    """Whole-job throughput of N independent replicas: every rank streams
+    bytes_per_rank per step; the job's step time is the slowest rank's."""
+    ms = max_over_ranks(ms_local, ws, device)
+    return ms, ws * bytes_per_rank / (ms * 1e-3) / 1e9
 
 
 def barrier(ws):
@@ -207,7 +215,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
-    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
+    ms_step, value = aggregate(cache_bytes, e0.elapsed_time(e1) / args.steps, ws)
     clk = clocks.stop()
     assert mla.get_error(s.ws) == mla.MLA_OK
 
@@ -236,7 +244,6 @@ def run_ours(args):
     del graph, g2
 
     tokens = wl.B * (wl.n_q if wl.mode == "decode" else wl.n_q)
-    value = ws * cache_bytes / (ms_step * 1e-3) / 1e9
     attn_avg_ms = attn_ms / max(1, attn_n)
     achieved = cache_bytes / (attn_avg_ms * 1e-3) / 1e9
     line = {

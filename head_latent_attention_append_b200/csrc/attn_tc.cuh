@@ -26,13 +26,15 @@
 // the same two numbers, so both see bit-identical scores and run identical
 // softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
 // half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
-// P [480, 512).  Shared memory: a 4-deep ring of per-page column groups
+// P [480, 512).  Shared memory: a 3-deep ring of per-page column groups
 // (<= 5 chunks of 64 keys x 64 columns, 128-byte swizzle, loaded by TMA) and
-// two 16 KB exchange buffers, filled by the peer with asynchronous remote
-// stores that complete on this CTA's mbarrier.
+// four 16 KB exchange buffers, filled by the peer with asynchronous remote
+// stores that complete on this CTA's mbarrier.  The softmax runs one page
+// behind the score MMA so the exchange round trip overlaps the next page.
 //
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (both
-// warp-uniform; one elected lane issues), warp 2 = TMEM allocator, warps 4-11 =
+// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = score-MMA issuer,
+// warp 3 = P*V-MMA issuer (all warp-uniform; one elected lane issues), warp 2 =
+// TMEM allocator, warps 4-11 =
 // two softmax / exchange / epilogue warpgroups (each owns half of the keys of
 // every row; thread r owns row r = TMEM lane r).  Every wait is bounded
 // (sm100::mbar_wait).
@@ -50,17 +52,18 @@ constexpr int THREADS = 384;
 constexpr int KT = 64;                        // keys per tile (one page)
 constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
 constexpr int MAX_OWN = 5;                    // chunks per CTA per page
-constexpr int GROUPS = 4;
+constexpr int GROUPS = 3;
+constexpr int XBUF = 4;                       // exchange buffers (the one-page lag needs 4)
 constexpr int GROUP_BYTES = MAX_OWN * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
 
 constexpr int OFF_G = 0;
 constexpr int OFF_X = OFF_G + GROUPS * GROUP_BYTES;
-constexpr int OFF_MH = OFF_X + 2 * X_BYTES;       // half-row maxima [2][2][128] fp32
+constexpr int OFF_MH = OFF_X + XBUF * X_BYTES;    // half-row maxima [2][2][128] fp32
 constexpr int OFF_LS = OFF_MH + 2 * 2 * 128 * 4;  // half-row sums [2][128] fp32
 constexpr int OFF_BAR = OFF_LS + 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * GROUPS + 2 + 7 + 4;
+constexpr int NUM_BARS = 2 * GROUPS + XBUF + 7 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to 1024
@@ -124,8 +127,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* g_full = bars;
   uint64_t* g_empty = bars + GROUPS;
-  uint64_t* x_full = bars + 2 * GROUPS;  // [2]
-  uint64_t* s_full = x_full + 2;
+  uint64_t* x_full = bars + 2 * GROUPS;  // [XBUF]
+  uint64_t* s_full = x_full + XBUF;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_full + 2;
   uint64_t* pv_done = s_full + 3;
@@ -151,15 +154,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&g_full[i], 1);
       mbar_init(&g_empty[i], 1);
     }
-    mbar_init(&x_full[0], 1);  // the receiver's expect_tx arrival + the peer's bytes
-    mbar_init(&x_full[1], 1);
+    for (int i = 0; i < XBUF; ++i) mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
     mbar_init(p_ready, 256);
     mbar_init(pv_done, 1);
     mbar_init(q_ready, 256);
     mbar_init(o_free, 256);
-    mbar_init(final_bar, 1);
+    mbar_init(final_bar, 2);  // one commit per issuer warp
     for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
     *abort_flag = 0;
     mbar_fence_init();
@@ -207,65 +209,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mbar_wait_warp(&g_full[q], (last / GROUPS) & 1, abort_flag, nullptr, 50000000ull, false);
       }
     }
-  } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
-    // Per tile: the partial score MMA of tile t, then the P*V MMA of tile t-1.
-    const uint32_t idS = idesc_bf16(128, 64, 0, 0);
-    const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------ MMA issuers
+    // Warp 1 issues the partial-score MMAs, warp 3 the P*V MMAs; each blocks
+    // only on its own inputs, and each tcgen05.commit tracks only the MMAs
+    // its own thread issued.
     const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q, tP = tbase + TM_P;
     const uint32_t sG = smem_u32(smem + OFF_G);
     uint32_t tg = 0, seg_k = 0;
     bool ok = true;
-    // P*V of the previous tile, issued right after the next score MMA.
-    auto issue_pv = [&](uint32_t gs, uint32_t tile_tg, bool first, uint32_t seg) -> bool {
-      if (!mbar_wait_warp(p_ready, tile_tg & 1, abort_flag, a.err)) return false;
-      if (first && seg > 0 && !mbar_wait_warp(o_free, (seg - 1) & 1, abort_flag, a.err)) return false;
-      tc_fence_after();
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk)
-          mma_ts(tO, tP + kk * 8, sdesc_sw128(sG + gs * GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
-                 (first && kk == 0) ? 0u : 1u);
-        tc_commit(pv_done);
-        tc_commit(&g_empty[gs]);
-      }
-      __syncwarp();
-      return true;
-    };
-    bool pv_pending = false, pv_first = false;
-    uint32_t pv_gs = 0, pv_tg = 0, pv_seg = 0;
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const Seg g = segs[si];
-      const int n = g.t_hi - g.t_lo;
-      if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
-      tc_fence_after();
-      for (int i = 0; i < n; ++i) {
-        if (tg > 0 && !(ok = mbar_wait_warp(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
-        const uint32_t gs = tg % GROUPS;
-        if (!(ok = mbar_wait_warp(&g_full[gs], (tg / GROUPS) & 1, abort_flag, a.err))) break;
+    if (warp == 1) {
+      const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
+        const int n = segs[si].t_hi - segs[si].t_lo;
+        if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
         tc_fence_after();
-        if (elect_one()) {
-          const uint32_t gb = sG + gs * GROUP_BYTES;
-          for (int q = 0; q < n_own; ++q) {
+        for (int i = 0; i < n; ++i) {
+          if (tg > 0 && !(ok = mbar_wait_warp(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
+          const uint32_t gs = tg % GROUPS;
+          if (!(ok = mbar_wait_warp(&g_full[gs], (tg / GROUPS) & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t gb = sG + gs * GROUP_BYTES;
+            for (int q = 0; q < n_own; ++q) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_ts(tS, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
-                     (q | k) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                mma_ts(tS, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
+                       (q | k) ? 1u : 0u);
+            }
+            tc_commit(s_full);
           }
-          tc_commit(s_full);
+          __syncwarp();
+          ++tg;
         }
-        __syncwarp();
-        if (pv_pending && !(ok = issue_pv(pv_gs, pv_tg, pv_first, pv_seg))) break;
-        pv_pending = true;
-        pv_first = (i == 0);
-        pv_gs = gs;
-        pv_tg = tg;
-        pv_seg = seg_k;
-        ++tg;
+        ++seg_k;
       }
-      ++seg_k;
+    } else {
+      const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
+        const int n = segs[si].t_hi - segs[si].t_lo;
+        for (int i = 0; i < n; ++i) {
+          if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
+          if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          const uint32_t gs = tg % GROUPS;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < KT / 16; ++kk)
+              mma_ts(tO, tP + kk * 8, sdesc_sw128(sG + gs * GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
+                     (i == 0 && kk == 0) ? 0u : 1u);
+            tc_commit(pv_done);
+            tc_commit(&g_empty[gs]);
+          }
+          __syncwarp();
+          ++tg;
+        }
+        ++seg_k;
+      }
     }
-    if (ok && pv_pending) ok = issue_pv(pv_gs, pv_tg, pv_first, pv_seg);
     if (elect_one()) tc_commit(final_bar);
     __syncwarp();
     mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
@@ -273,8 +274,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // ------------------------------- softmax, score exchange and epilogue
     // Two warpgroups: WG h (warps 4+4h .. 7+4h) owns keys [32h, 32h + 32) of
     // every row; thread r of a WG owns row r (= TMEM lane r).  The two threads
-    // of a row meet at a 64-thread named barrier (their warps share a lane
-    // quarter) to agree on the row maximum.
+    // of a row agree on the row maximum through a 64-arrival mbarrier (their
+    // warps share a lane quarter).  The softmax runs one page behind the
+    // score: "send" reads page t's partial score and passes it to the peer,
+    // then "finish" completes page t-1, whose peer half has had a page's time
+    // to arrive.
     const int h = warp >= 8 ? 1 : 0;
     const int r = tid - 128 - 128 * h;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -287,22 +291,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     float* mh = reinterpret_cast<float*>(smem + OFF_MH);
     float* ls = reinterpret_cast<float*>(smem + OFF_LS);
     const uint32_t peer_x = map_peer(smem_u32(sX), peer);
-    const uint32_t peer_xbar0 = map_peer(smem_u32(&x_full[0]), peer);
-    const uint32_t peer_xbar1 = map_peer(smem_u32(&x_full[1]), peer);
+    const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
     const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
     const int hc0 = h * (dh / 64), hc1 = hc0 + dh / 64;  // this WG's 32-column chunks of O
-    uint32_t tg = 0;
     bool ok = true;
 
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
+      return __all_sync(0xffffffffu, r_ok);
+    };
     // Meeting point of the two threads of a row (bounded, like every wait).
     auto pair_sync = [&]() -> bool {
       mbar_arrive(pair_bar);
       bool r_ok = mbar_wait(pair_bar, pair_phase & 1, abort_flag, a.err);
       ++pair_phase;
-      return __all_sync(0xffffffffu, r_ok);
-    };
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
       return __all_sync(0xffffffffu, r_ok);
     };
     // Row r of this CTA's Q slice (chunks c_lo .. c_lo + n_own - 1) into TMEM;
@@ -328,150 +330,126 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_arrive(q_ready);
     };
 
-    if (seg_lo < seg_hi) load_q(segs[seg_lo].rb);
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
+    float m_used = -INFINITY, l = 0.f;
+    // Finish tile i of segment si (global tile tgf): combine the two fp16
+    // partial scores, softmax, P into TMEM; the segment's epilogue after its
+    // last tile.
+    auto finish = [&](int si, int i, uint32_t tgf, const uint32_t (&mine)[16]) -> bool {
       const Seg g = segs[si];
       const int rb = g.rb;
+      const int t = g.t_lo + i;
       const int nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
-      const int n = g.t_hi - g.t_lo;
-      float m_used = -INFINITY, l = 0.f;
-      for (int i = 0; i < n; ++i) {
-        const int t = g.t_lo + i;
-        const uint32_t xb = tg & 1;
-        if (!(ok = wait_all(s_full, tg & 1))) break;
+      const uint32_t xb = tgf % XBUF;
+      if (!wait_all(&x_full[xb], (tgf / XBUF) & 1)) return false;
+      float s[32];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(sX + xb * X_BYTES + r * 128 + h * 64);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 pv = src[u];
+          const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = unpack_half2(mine[4 * u + e]);
+            const float2 y = unpack_half2(pw[e]);
+            s[8 * u + 2 * e] = x.x + y.x;
+            s[8 * u + 2 * e + 1] = x.y + y.y;
+          }
+        }
+      }
+      const int valid_all = min(KT, nkeys - t * KT);
+      const int valid = valid_all - 32 * h;  // valid keys among this WG's 32
+      if (valid < 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j >= valid) s[j] = -INFINITY;
+      }
+      float mt;
+      {
+        float mx[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
+#pragma unroll
+        for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+        float* slot = mh + (tgf & 1) * 256;
+        slot[h * 128 + r] = mx[0];
+        if (!pair_sync()) return false;
+        mt = fmaxf(slot[r], slot[128 + r]);
+      }
+      // Running max with lazy rescaling: O and l stay relative to m_used
+      // until a tile's max exceeds it by more than 2^8.
+      bool resc = false;
+      float scale = 1.f;
+      if (i == 0) {
+        m_used = mt;
+        l = 0.f;
+      } else if (mt > m_used + 8.f) {
+        scale = fast_exp2(m_used - mt);
+        m_used = mt;
+        resc = true;
+      }
+      uint32_t pk[16];
+      float psum;
+      {
+        float ps[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          ps[u] = 0.f;
+          pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u]);
+        }
+#pragma unroll
+        for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
+        psum = ps[0];
+      }
+      // The previous P*V must be done before P is overwritten or O rescaled.
+      if (tgf > 0) {
+        if (!wait_all(pv_done, (tgf - 1) & 1)) return false;
         tc_fence_after();
-        // Own partial score (this WG's 32 keys), rounded to fp16; the same
-        // values go to the peer.
-        uint32_t own[16];
-        {
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        for (int cc = hc0; cc < hc1; ++cc) {
           uint32_t v[32];
-          tmem_ld32(tS, v);
+          tmem_ld32(tO + cc * 32, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) own[j] = pack_half2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
+          tmem_st32(tO + cc * 32, v);
         }
-        tc_fence_before();
-        mbar_arrive(s_free);
-        {
-          const uint32_t dst = peer_x + xb * X_BYTES + r * 128 + h * 64;
-          const uint32_t pbar = xb ? peer_xbar1 : peer_xbar0;
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_async_peer_v4(dst + u * 16, make_uint4(own[4 * u], own[4 * u + 1], own[4 * u + 2], own[4 * u + 3]),
-                             pbar);
-        }
-        if (h == 0 && r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
-        if (!(ok = wait_all(&x_full[xb], (tg >> 1) & 1))) break;
-        float s[32];
-        {
-          const uint4* src = reinterpret_cast<const uint4*>(sX + xb * X_BYTES + r * 128 + h * 64);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 pv = src[u];
-            const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 mine = unpack_half2(own[4 * u + e]);
-              const float2 theirs = unpack_half2(pw[e]);
-              s[8 * u + 2 * e] = mine.x + theirs.x;
-              s[8 * u + 2 * e + 1] = mine.y + theirs.y;
-            }
-          }
-        }
-        const int valid = min(KT, nkeys - t * KT) - 32 * h;  // valid keys among this WG's 32
-        if (valid < 32) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j >= valid) s[j] = -INFINITY;
-        }
-        float mt;
-        {
-          float mx[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
-#pragma unroll
-          for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-            for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-          float* slot = mh + (tg & 1) * 256;
-          slot[h * 128 + r] = mx[0];
-          ok = pair_sync();
-          mt = fmaxf(slot[r], slot[128 + r]);
-        }
-        if (!ok) break;
-        // Running max with lazy rescaling: O and l stay relative to m_used
-        // until a tile's max exceeds it by more than 2^8.
-        bool resc = false;
-        float scale = 1.f;
-        if (i == 0) {
-          m_used = mt;
-          l = 0.f;
-        } else if (mt > m_used + 8.f) {
-          scale = fast_exp2(m_used - mt);
-          m_used = mt;
-          resc = true;
-        }
-        uint32_t pk[16];
-        float psum;
-        {
-          float ps[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            ps[u] = 0.f;
-            pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u]);
-          }
-#pragma unroll
-          for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-            for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
-          psum = ps[0];
-        }
-        if (i > 0) {
-          if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
-          tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, resc)) {
-          for (int cc = hc0; cc < hc1; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tO + cc * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
-            tmem_st32(tO + cc * 32, v);
-          }
-          l *= scale;
-        }
-        tmem_st16(tP, pk);
-        tmem_st_wait();
-        l += psum;
-        const int valid_all = min(KT, nkeys - t * KT);
-        if (valid_all < KT) {
-          // Keys past the end: P is 0 there, but 0 * NaN would still poison O,
-          // so clear those rows of this tile's latent chunks.
-          uint8_t* gb = sG + (tg % GROUPS) * GROUP_BYTES;
-          const int rows = KT - valid_all, units = rows * 8 * npv;
-          for (int x = r + 128 * h; x < units; x += 256) {
-            const int q = x / (rows * 8), rem = x - q * rows * 8;
-            *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        mbar_arrive(p_ready);
-        ++tg;
+        l *= scale;
       }
-      if (!ok) break;
-      if (si + 1 < seg_hi) load_q(segs[si + 1].rb);
-      if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
+      tmem_st16(tP, pk);
+      tmem_st_wait();
+      l += psum;
+      if (valid_all < KT) {
+        // Keys past the end: P is 0 there, but 0 * NaN would still poison O,
+        // so clear those rows of this tile's latent chunks.
+        uint8_t* gb = sG + (tgf % GROUPS) * GROUP_BYTES;
+        const int rows = KT - valid_all, units = rows * 8 * npv;
+        for (int x = r + 128 * h; x < units; x += 256) {
+          const int q = x / (rows * 8), rem = x - q * rows * 8;
+          *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      if (i + 1 < g.t_hi - g.t_lo) return true;
+
+      // ---- epilogue of the segment ----
+      if (!wait_all(pv_done, tgf & 1)) return false;
       tc_fence_after();
       // Row sum: both halves add the two partial sums in the same order.
       ls[h * 128 + r] = l;
-      if (!(ok = pair_sync())) break;
+      if (!pair_sync()) return false;
       const float lrow = ls[r] + ls[128 + r];
-      if (!(ok = pair_sync())) break;  // both have read before the next segment's write
-      // Epilogue: a whole row block is normalised into obar (bf16); a piece of
-      // a split row block leaves its unnormalised sum and (m, l) in its slot.
+      if (!pair_sync()) return false;  // both have read before the next write
+      // A whole row block is normalised into obar (bf16); a piece of a split
+      // row block leaves its unnormalised sum and (m, l) in its slot.
       const bool whole = g.slot < 0;
       const float inv = 1.f / lrow;
       for (int cc = hc0; cc < hc1; ++cc) {
@@ -506,7 +484,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(o_free);
+      return true;
+    };
+
+    if (seg_lo < seg_hi) load_q(segs[seg_lo].rb);
+    uint32_t own[16];
+    int fin_si = -1, fin_i = 0;
+    uint32_t fin_tg = 0, tg = 0;
+    for (int si = seg_lo; si < seg_hi && ok; ++si) {
+      const int n = segs[si].t_hi - segs[si].t_lo;
+      for (int i = 0; i < n && ok; ++i) {
+        // ---- send: read page tg's partial score, pass it to the peer ----
+        const uint32_t xb = tg % XBUF;
+        if (!(ok = wait_all(s_full, tg & 1))) break;
+        tc_fence_after();
+        uint32_t cur[16];
+        {
+          uint32_t v[32];
+          tmem_ld32(tS, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) cur[j] = pack_half2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(s_free);
+        {
+          const uint32_t dst = peer_x + xb * X_BYTES + r * 128 + h * 64;
+          const uint32_t pbar = peer_xbar + xb * 8;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            st_async_peer_v4(dst + u * 16, make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]),
+                             pbar);
+        }
+        if (h == 0 && r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
+        // The segment's scores are all read after its last page, so the next
+        // segment's Q may replace this one's.
+        if (i + 1 == n && si + 1 < seg_hi) load_q(segs[si + 1].rb);
+        // ---- finish the previous page ----
+        if (fin_si >= 0 && !(ok = finish(fin_si, fin_i, fin_tg, own))) break;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) own[j] = cur[j];
+        fin_si = si;
+        fin_i = i;
+        fin_tg = tg;
+        ++tg;
+      }
     }
+    if (ok && fin_si >= 0) ok = finish(fin_si, fin_i, fin_tg, own);
   }
 
   tc_fence_before();

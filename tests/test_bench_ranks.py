@@ -1,0 +1,55 @@
+"""bench.py's multi-replica accounting on two gloo ranks (CPU): the step time
+is the slowest rank's, and the job's value sums the ranks' bytes."""
+import os
+import socket
+import sys
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, ws, port, q):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    ms_local = [2.0, 3.0][rank]
+    ms, value = bench.aggregate(1_000_000_000, ms_local, ws, device="cpu")
+    q.put((rank, ms, value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_replicas_report_slowest_time_and_summed_bytes():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for _, ms, value in res:
+        assert ms == 3.0
+        assert value == pytest.approx(2 * 1e9 / 3e-3 / 1e9)
+
+
+def test_single_rank_is_passthrough():
+    sys.path.insert(0, ROOT)
+    import bench
+    ms, value = bench.aggregate(604_053_504, 0.5, 1)
+    assert ms == 0.5 and value == pytest.approx(604_053_504 / 0.5e-3 / 1e9)
