@@ -21,8 +21,8 @@
 //   rank 1: latent columns [d_c/2, d_c) and the RoPE key columns.
 // Each CTA streams only its own columns of every page (no byte is read twice),
 // computes the partial score over them (all of its Q slice is the TMEM A
-// operand), and sends the partial, rounded to fp16, to its peer through
-// distributed shared memory.  Both CTAs add the two fp16 partials in fp32 --
+// operand), and sends the partial, rounded to bf16, to its peer through
+// distributed shared memory.  Both CTAs add the two bf16 partials in fp32 --
 // the same two numbers, so both see bit-identical scores and run identical
 // softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
 // half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
@@ -34,13 +34,10 @@
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = score-MMA issuer,
 // warp 3 = P*V-MMA issuer (all warp-uniform; one elected lane issues), warp 2 =
-// TMEM allocator, warps 4-11 =
-// two softmax / exchange / epilogue warpgroups (each owns half of the keys of
-// every row; thread r owns row r = TMEM lane r).  Every wait is bounded
-// (sm100::mbar_wait).
+// TMEM allocator, warps 4-11 = two softmax / exchange / epilogue warpgroups
+// (each owns half of the keys of every row; thread r owns row r = TMEM lane
+// r).  Every wait is bounded (sm100::mbar_wait).
 #pragma once
-#include <cuda_fp16.h>
-
 #include "attn_simt.cuh"
 #include "sm100.cuh"
 
@@ -55,7 +52,7 @@ constexpr int MAX_OWN = 5;                    // chunks per CTA per page
 constexpr int GROUPS = 3;
 constexpr int XBUF = 4;                       // exchange buffers (the one-page lag needs 4)
 constexpr int GROUP_BYTES = MAX_OWN * CHUNK_BYTES;
-constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
+constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
 
 constexpr int OFF_G = 0;
@@ -111,13 +108,14 @@ __device__ __forceinline__ void st_async_peer_v4(uint32_t addr, uint4 v, uint32_
                "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
                : "memory");
 }
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
+// Partial scores travel between the CTAs as bf16 pairs: packing is one
+// conversion, unpacking is two integer ops (no conversion-pipe work).
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float2 unpack_half2(uint32_t u) {
-  __half2 h = *reinterpret_cast<__half2*>(&u);
-  return __half22float2(h);
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -331,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
 
     float m_used = -INFINITY, l = 0.f;
-    // Finish tile i of segment si (global tile tgf): combine the two fp16
+    // Finish tile i of segment si (global tile tgf): combine the two bf16
     // partial scores, softmax, P into TMEM; the segment's epilogue after its
     // last tile.
     auto finish = [&](int si, int i, uint32_t tgf, const uint32_t (&mine)[16]) -> bool {
@@ -350,8 +348,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_half2(mine[4 * u + e]);
-            const float2 y = unpack_half2(pw[e]);
+            const float2 x = unpack_bf16x2(mine[4 * u + e]);
+            const float2 y = unpack_bf16x2(pw[e]);
             s[8 * u + 2 * e] = x.x + y.x;
             s[8 * u + 2 * e + 1] = x.y + y.y;
           }
@@ -504,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tmem_ld32(tS, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) cur[j] = pack_half2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          for (int j = 0; j < 16; ++j) cur[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
         }
         tc_fence_before();
         mbar_arrive(s_free);
