@@ -1,15 +1,17 @@
 #!/usr/bin/env python
-"""Benchmark: one decode step of multi-head latent attention on the paged
-latent cache (append the new tokens, then attend), on the DeepSeek-V2-like
-workload (B=64, n_h=128, d_c=512, d_r=64, 8192 cached tokens + 1 new token per
-sequence, bf16), timed on the device with CUDA events.
+"""Benchmark: one step of multi-head latent attention on the paged latent
+cache -- append the new tokens, then attend -- timed on the device with CUDA
+events.  The default workload is the DeepSeek-V2-like decode (B=64, n_h=128,
+d_c=512, d_r=64, 8192 cached tokens + 1 new token per sequence, bf16); the
+other named workloads (synth.WORKLOADS) run with --workload.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  Multi-GPU runs are independent replicas (the
-path shards by sequence; there is no collective on the data path), so
-`value` is the sum over ranks of the bytes each rank streamed divided by the
-slowest rank's time.
+Prints one JSON line (rank 0).  `value` is latent-cache GB/s (each sequence's
+cache counted once per step) for decode workloads and attention TFLOP/s for
+prefill.  Multi-GPU runs are independent replicas (the path shards by
+sequence; there is no collective on the data path), so `value` is the sum over
+ranks of what each rank processed divided by the slowest rank's time.
 """
 import argparse
 import json
@@ -103,11 +105,12 @@ def max_over_ranks(x: float, ws: int, device: str = "cuda") -> float:
     return float(t.item())
 
 
-def aggregate(bytes_per_rank: int, ms_local: float, ws: int, device: str = "cuda"):
-    """Whole-job throughput of N independent replicas: every rank streams
-    bytes_per_rank per step; the job's step time is the slowest rank's."""
+def aggregate(units_per_rank: float, ms_local: float, ws: int, device: str = "cuda", scale: float = 1e9):
+    """Whole-job throughput of N independent replicas: every rank processes
+    units_per_rank (bytes, or flops) per step; the job's step time is the
+    slowest rank's.  Returns (ms, units / s / scale)."""
     ms = max_over_ranks(ms_local, ws, device)
-    return ms, ws * bytes_per_rank / (ms * 1e-3) / 1e9
+    return ms, ws * units_per_rank / (ms * 1e-3) / scale
 
 
 def barrier(ws):
@@ -116,52 +119,111 @@ def barrier(ws):
         dist.barrier()
 
 
-def oracle_sample(name: str):
-    """Times the fp64 oracle on one sequence of the workload (its full
-    history and its new tokens): returns (seconds, cache bytes, tokens)."""
+PREFILL_SAMPLE_TOKENS = 1024   # causal prefix of one sequence per oracle prefill sample
+
+
+def blas_threads() -> int:
+    """Threads the oracle's BLAS actually runs with."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(name: str, k: int = 0):
+    """Times the fp64 oracle on one bounded unit of the workload: the k-th
+    sequence (in a seeded order) of a decode workload, with its whole history
+    and its new tokens, or the causal prefix of PREFILL_SAMPLE_TOKENS tokens
+    of one sequence of a prefill workload.  Returns a dict with the seconds,
+    the unique cache bytes, the attention flops, the query tokens and a
+    description."""
     import numpy as np
     import oracle as O
     from head_latent_attention_append_b200 import synth
     wl = synth.WORKLOADS[name]
     kv = synth.kv_lengths(wl)
-    b = int(np.argsort(kv)[len(kv) // 2])
+    med = int(np.argsort(kv)[len(kv) // 2])   # the median-length sequence first, then a seeded order
+    order = [med] + [int(i) for i in np.random.default_rng(wl.wid).permutation(len(kv)) if i != med]
+    b = order[k % len(order)]
     hw = synth.make_weights(wl)
     dims = O.Dims(wl.n_h, wl.d_h, wl.d_v, wl.d_c, wl.d_r, wl.d_model, wl.d_cq, wl.rope_base)
     w = O.Weights(**hw.as_dict())
-    L = int(kv[b])
+    if wl.mode == "prefill":
+        L = nq = min(PREFILL_SAMPLE_TOKENS, int(kv[b]))
+        what = f"causal prefix of {L} tokens of sequence {b} of {wl.B} (S={int(kv[b])})"
+    else:
+        L, nq = int(kv[b]), wl.n_q
+        what = f"sequence {b} of {wl.B} ({L} keys, {nq} new token(s))"
     H = synth.make_hidden(wl, b, L)
     t0 = time.perf_counter()
-    O.mla_decode(dims, w, H, wl.n_q)
+    O.mla_decode(dims, w, H, nq)
     dt = time.perf_counter() - t0
     esz = 2 if wl.dtype == "bf16" else 4
-    keys = sum(L - wl.n_q + 1 + q for q in range(wl.n_q))
-    return dt, keys * wl.d_cr * esz, wl.n_q, f"1 of {wl.B} sequences ({L} keys, {wl.n_q} new token(s))"
+    pairs = sum(L - nq + 1 + q for q in range(nq))
+    return {"seconds": dt, "bytes": L * wl.d_cr * esz, "flops": pairs * wl.n_h * (2 * wl.d_cr + 2 * wl.d_c),
+            "tokens": nq, "what": what}
+
+
+def metric_of(mode: str, nbytes: float, flops: float, seconds: float):
+    """The workload's headline figure: latent-cache GB/s for decode, attention
+    TFLOP/s for prefill."""
+    if mode == "prefill":
+        return flops / seconds / 1e12, "TFLOP/s"
+    return nbytes / seconds / 1e9, "GB/s"
+
+
+def cpu_baseline(name: str, min_seconds: float = 10.0, max_samples: int = 16):
+    """The oracle on successive bounded samples until about min_seconds of
+    CPU work; returns the line's cpu_baseline object."""
+    from head_latent_attention_append_b200 import synth
+    mode = synth.WORKLOADS[name].mode
+    tot = {"seconds": 0.0, "bytes": 0, "flops": 0, "tokens": 0}
+    whats = []
+    k = 0
+    while k < max_samples and (k == 0 or tot["seconds"] < min_seconds):
+        r = oracle_sample(name, k)
+        for key in tot:
+            tot[key] += r[key]
+        whats.append(r["what"])
+        k += 1
+    val, unit = metric_of(mode, tot["bytes"], tot["flops"], tot["seconds"])
+    return {"value": val, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{k} sample(s), {tot['seconds']:.1f} s of fp64 oracle work: " + "; ".join(whats),
+            "seconds": tot["seconds"], "tokens_per_s": tot["tokens"] / tot["seconds"]}
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, one bounded sample
+    per step, on the same metric and unit as the GPU line."""
+    from head_latent_attention_append_b200 import synth
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cores = os.cpu_count()
-    for _ in range(args.warmup):
-        oracle_sample(args.workload)
-    tot_t = tot_b = tot_tok = 0.0
-    sample = ""
-    for _ in range(args.steps):
-        dt, nb, ntok, sample = oracle_sample(args.workload)
-        tot_t += dt
-        tot_b += nb
-        tot_tok += ntok
-    val = tot_b / tot_t / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+    mode = synth.WORKLOADS[args.workload].mode
+    for i in range(args.warmup):
+        oracle_sample(args.workload, i)
+    tot = {"seconds": 0.0, "bytes": 0, "flops": 0, "tokens": 0}
+    whats = []
+    for i in range(args.steps):
+        r = oracle_sample(args.workload, i)
+        for key in tot:
+            tot[key] += r[key]
+        whats.append(r["what"])
+    val, unit = metric_of(mode, tot["bytes"], tot["flops"], tot["seconds"])
+    sample = f"one bounded sample per step ({whats[0]}{', ...' if len(whats) > 1 else ''})"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot["seconds"] / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": args.workload},
-            "tokens_per_s": tot_tok / tot_t,
-            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": f"per step: {sample}"},
-            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "tokens_per_s": tot["tokens"] / tot["seconds"],
+            "cpu_baseline": {"value": val, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -173,8 +235,13 @@ def run_ours(args):
     peaks = load_peaks()
     s = workload.setup(args.workload, device=f"cuda:{local}", checked_count=0, check_all=False)
     wl = s.wl
-    cache_bytes = s.cache_bytes_read()
+    prefill = wl.mode == "prefill"
+    unique_bytes = s.cache_bytes_unique()    # the latent cache, each key once
+    streamed_bytes = s.cache_bytes_read()    # what the kernel streams (once per query row block)
     flops = s.attention_flops()
+    # Headline units per step: cache bytes (decode, GB/s) or attention flops
+    # (prefill, TFLOP/s).
+    units, scale, unit = (flops, 1e12, "TFLOP/s") if prefill else (unique_bytes, 1e9, "GB/s")
     stream = torch.cuda.current_stream()
 
     # Launch accounting for one step.
@@ -215,7 +282,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
-    ms_step, value = aggregate(cache_bytes, e0.elapsed_time(e1) / args.steps, ws)
+    ms_step, value = aggregate(units, e0.elapsed_time(e1) / args.steps, ws, scale=scale)
     clk = clocks.stop()
     assert mla.get_error(s.ws) == mla.MLA_OK
 
@@ -243,34 +310,46 @@ def run_ours(args):
     ms_e2e = max_over_ranks(e2.elapsed_time(e3) / args.steps, ws)
     del graph, g2
 
-    tokens = wl.B * (wl.n_q if wl.mode == "decode" else wl.n_q)
+    tokens = wl.B * wl.n_q
     attn_avg_ms = attn_ms / max(1, attn_n)
-    achieved = cache_bytes / (attn_avg_ms * 1e-3) / 1e9
+    hbm_gbs = unique_bytes / (attn_avg_ms * 1e-3) / 1e9
+    tc_tflops = flops / (attn_avg_ms * 1e-3) / 1e12
+    # The attention kernel runs inside a step of several kernels, back to
+    # back: the sustained tensor peak applies.
+    tc_peak = peaks["bf16_tflops_sustained"]
+    hbm_roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm_gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": unique_bytes}
+    tc_roof = {"bound": "tensor", "achieved": tc_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+               "frac": tc_tflops / tc_peak, "algorithmic_flops_per_launch": flops,
+               "peak_kind": "bf16 sustained"}
+    main_roof, other_roof = (tc_roof, hbm_roof) if prefill else (hbm_roof, tc_roof)
+    roofline = dict(main_roof, traffic=None, kernel="latent attention (split-KV)", peak_src=peaks["src"],
+                    avg_kernel_ms=attn_avg_ms, streamed_cache_bytes_per_launch=streamed_bytes,
+                    other_roof=other_roof)
+    l2_note = (f"inputs larger than L2: {wl.B * wl.n_q * wl.d_model * 2 / 1e6:.0f} MB of hidden states in and "
+               f"{s.out.numel() * 4 / 1e6:.0f} MB out per step" if prefill else
+               f"inputs larger than L2: {unique_bytes / 1e6:.0f} MB of latent cache read per step")
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "n_q": wl.n_q, "kv_len": int(s.kv_len_host.max()),
                    "n_h": wl.n_h, "d_c": wl.d_c, "d_r": wl.d_r, "d_model": wl.d_model, "d_cq": wl.d_cq,
                    "page_size": synth.PAGE_SIZE, "parallelism": f"replicas{ws}" if ws > 1 else "single",
-                   "l2": f"inputs larger than L2: {cache_bytes / 1e6:.0f} MB of cache read per step",
+                   "l2": l2_note,
                    "timing": "CUDA graph of one step, replayed; CUDA events on the launching stream"},
         "tokens_per_s": ws * tokens / (ms_step * 1e-3),
+        "cache_gbs": ws * unique_bytes / (ms_step * 1e-3) / 1e9,
         "attention_tflops": ws * flops / (ms_step * 1e-3) / 1e12,
-        "roofline": {"bound": "hbm", "kernel": "latent attention (split-KV)", "achieved": achieved,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": None, "peak_src": peaks["src"], "avg_kernel_ms": attn_avg_ms,
-                     "algorithmic_bytes_per_launch": cache_bytes},
-        "e2e": {"value": ws * cache_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+        "roofline": roofline,
+        "e2e": {"value": ws * units / (ms_e2e * 1e-3) / scale, "unit": unit,
                 "h2d_bytes_per_step": s.h_new.numel() * s.h_new.element_size(),
                 "d2h_bytes_per_step": s.out.numel() * s.out.element_size(), "ms_per_step": ms_e2e},
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        dt, nb, _, sample = oracle_sample(args.workload)
-        line["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
-                                "sample": sample, "seconds": dt}
+        line["cpu_baseline"] = cpu_baseline(args.workload)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -28,9 +28,12 @@
 // half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
 // P [480, 512).  Shared memory: a 3-deep ring of per-page column groups
 // (<= 5 chunks of 64 keys x 64 columns, 128-byte swizzle, loaded by TMA) and
-// four 16 KB exchange buffers, filled by the peer with asynchronous remote
-// stores that complete on this CTA's mbarrier.  The softmax runs one page
-// behind the score MMA so the exchange round trip overlaps the next page.
+// five 16 KB exchange buffers, filled by the peer with bulk copies (one per
+// softmax warp per page, staged in a local 16 KB block) that complete on this
+// CTA's mbarrier; there are enough buffers that the pipeline itself keeps the
+// peer from overwriting an unread one (see XBUF).
+// The softmax runs one page behind the score MMA so the exchange round trip
+// overlaps the next page.
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = score-MMA issuer,
 // warp 3 = P*V-MMA issuer (all warp-uniform; one elected lane issues), warp 2 =
@@ -49,15 +52,23 @@ constexpr int THREADS = 384;
 constexpr int KT = 64;                        // keys per tile (one page)
 constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
 constexpr int MAX_OWN = 5;                    // chunks per CTA per page
-constexpr int GROUPS = 3;
-constexpr int XBUF = 4;                       // exchange buffers (the one-page lag needs 4)
+constexpr int GROUPS = 3;                     // page groups in flight
+constexpr int XBUF = 5;                       // exchange buffers per CTA
+// A CTA refills the peer's exchange buffer for page t + XBUF only after its
+// own page group of page t + XBUF - GROUPS has been consumed by P*V, which
+// needs the peer's partial of that page, which the peer sends after reading
+// page t's buffer whenever t + XBUF - GROUPS >= t + 2 (the softmax runs one
+// page behind).  So no partial can overwrite one that is still unread, with
+// no extra barrier.
+static_assert(XBUF >= GROUPS + 2, "exchange buffers must outlast the page ring by the softmax lag + 1");
 constexpr int GROUP_BYTES = MAX_OWN * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
 
 constexpr int OFF_G = 0;
 constexpr int OFF_X = OFF_G + GROUPS * GROUP_BYTES;
-constexpr int OFF_MH = OFF_X + XBUF * X_BYTES;    // half-row maxima [2][2][128] fp32
+constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
+constexpr int OFF_MH = OFF_XS + X_BYTES;          // half-row maxima [2][2][128] fp32
 constexpr int OFF_LS = OFF_MH + 2 * 2 * 128 * 4;  // half-row sums [2][128] fp32
 constexpr int OFF_BAR = OFF_LS + 2 * 128 * 4;
 constexpr int NUM_BARS = 2 * GROUPS + XBUF + 7 + 4;
@@ -100,14 +111,21 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// Asynchronous 16-byte store into a peer CTA's shared memory; its bytes count
-// toward the transaction count of the peer's mbarrier `bar_cluster_addr`.
-__device__ __forceinline__ void st_async_peer_v4(uint32_t addr, uint4 v, uint32_t bar_cluster_addr) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   addr),
-               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
-               : "memory");
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
+// a peer CTA's, completing as transaction bytes on the peer's mbarrier
+// `bar_cluster_addr`.  One copy carries what would otherwise be many small
+// remote stores, each with its own transaction-count update at the peer.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster_addr, uint32_t src_smem, uint32_t bytes,
+                                                  uint32_t bar_cluster_addr) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster_addr),
+      "r"(src_smem), "r"(bytes), "r"(bar_cluster_addr)
+      : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the sources of this thread's committed bulk copies have been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Partial scores travel between the CTAs as bf16 pairs: packing is one
 // conversion, unpacking is two integer ops (no conversion-pipe work).
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -118,6 +136,15 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
+// Byte offset, in an exchange tile, of 16-byte piece u (0..3) of the 32
+// partial scores that thread r of warpgroup h owns.  Layout [h][r][64 bytes],
+// so each warp's 32 rows form one contiguous 2 KB block (one bulk copy); the
+// pieces are XOR-swizzled by (r >> 1) so that the eight rows a quarter-warp
+// touches at once fall in eight different bank groups.
+__device__ __forceinline__ uint32_t x_off(int r, int h, int u) {
+  return (uint32_t)(h * (X_BYTES / 2) + r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -125,7 +152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* g_full = bars;
   uint64_t* g_empty = bars + GROUPS;
-  uint64_t* x_full = bars + 2 * GROUPS;  // [XBUF]
+  uint64_t* x_full = bars + 2 * GROUPS;  // [XBUF] the peer's partial has landed here
   uint64_t* s_full = x_full + XBUF;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_full + 2;
@@ -177,19 +204,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
+    // Metadata loads run one step ahead: the next segment while this one
+    // streams, the next page id while this page waits for its ring slot.
     uint32_t cnt = 0;
-    bool ok = true;
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const Seg g = segs[si];
-      const int seq = g.rb / a.n_q;
-      for (int t = g.t_lo; t < g.t_hi; ++t) {
-        int page = a.page_table[(long long)seq * a.max_pages + t];
+    if (seg_lo < seg_hi) {
+      int si = seg_lo;
+      Seg g = segs[si];
+      Seg gn = si + 1 < seg_hi ? segs[si + 1] : g;
+      int t = g.t_lo;
+      int page_n = a.page_table[(long long)(g.rb / a.n_q) * a.max_pages + t];
+      bool more = true;
+      while (more) {
+        int page = page_n;
+        if (++t >= g.t_hi) {
+          if (++si < seg_hi) {
+            g = gn;
+            if (si + 1 < seg_hi) gn = segs[si + 1];
+            t = g.t_lo;
+          } else {
+            more = false;
+          }
+        }
+        if (more) page_n = a.page_table[(long long)(g.rb / a.n_q) * a.max_pages + t];
+        const uint32_t gs = cnt % GROUPS;
+        if (!mbar_wait_warp(&g_empty[gs], ((cnt / GROUPS) & 1) ^ 1, abort_flag, a.err)) break;
         if (page < 0 || page >= a.num_pages) {
           if (rank == 0 && elect_one()) flag_error(a.err, kErrBounds);
           page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
         }
-        const uint32_t gs = cnt % GROUPS;
-        if (!(ok = mbar_wait_warp(&g_empty[gs], ((cnt / GROUPS) & 1) ^ 1, abort_flag, a.err))) break;
         if (elect_one()) {
           mbar_arrive_expect_tx(&g_full[gs], n_own * CHUNK_BYTES);
           for (int q = 0; q < n_own; ++q)
@@ -218,8 +260,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     bool ok = true;
     if (warp == 1) {
       const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+      Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
       for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const int n = segs[si].t_hi - segs[si].t_lo;
+        const Seg g = gn;
+        if (si + 1 < seg_hi) gn = segs[si + 1];  // in flight while this segment runs
+        const int n = g.t_hi - g.t_lo;
         if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
         tc_fence_after();
         for (int i = 0; i < n; ++i) {
@@ -244,8 +289,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
     } else {
       const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
+      Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
       for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const int n = segs[si].t_hi - segs[si].t_lo;
+        const Seg g = gn;
+        if (si + 1 < seg_hi) gn = segs[si + 1];
+        const int n = g.t_hi - g.t_lo;
         for (int i = 0; i < n; ++i) {
           if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
           if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
@@ -286,6 +334,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t pair_phase = 0;
     uint8_t* sG = smem + OFF_G;
     uint8_t* sX = smem + OFF_X;
+    uint8_t* sXS = smem + OFF_XS;
+    const int lane = tid & 31;
     float* mh = reinterpret_cast<float*>(smem + OFF_MH);
     float* ls = reinterpret_cast<float*>(smem + OFF_LS);
     const uint32_t peer_x = map_peer(smem_u32(sX), peer);
@@ -329,22 +379,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
 
     float m_used = -INFINITY, l = 0.f;
-    // Finish tile i of segment si (global tile tgf): combine the two bf16
+    // Finish tile i of segment g (global tile tgf): combine the two bf16
     // partial scores, softmax, P into TMEM; the segment's epilogue after its
     // last tile.
-    auto finish = [&](int si, int i, uint32_t tgf, const uint32_t (&mine)[16]) -> bool {
-      const Seg g = segs[si];
+    auto finish = [&](const Seg& g, int i, uint32_t tgf, const uint32_t (&mine)[16]) -> bool {
       const int rb = g.rb;
       const int t = g.t_lo + i;
-      const int nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
+      const int nkeys = g.nkeys;
       const uint32_t xb = tgf % XBUF;
-      if (!wait_all(&x_full[xb], (tgf / XBUF) & 1)) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&x_full[xb], (tgf / XBUF) & 1, abort_flag, a.err, 2000000000ull, true,
+                                             true)))
+        return false;
       float s[32];
       {
-        const uint4* src = reinterpret_cast<const uint4*>(sX + xb * X_BYTES + r * 128 + h * 64);
+        const uint8_t* src = sX + xb * X_BYTES;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint4 pv = src[u];
+          const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, h, u));
           const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -485,12 +536,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       return true;
     };
 
-    if (seg_lo < seg_hi) load_q(segs[seg_lo].rb);
+    // Segment metadata stays in registers, the next segment's loaded a
+    // segment ahead, so no global load sits on a page's critical path.
+    Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
+    Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
+    if (seg_lo < seg_hi) load_q(g_cur.rb);
     uint32_t own[16];
-    int fin_si = -1, fin_i = 0;
+    Seg fin_g{};
+    bool fin_any = false;
+    int fin_i = 0;
     uint32_t fin_tg = 0, tg = 0;
     for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const int n = segs[si].t_hi - segs[si].t_lo;
+      const Seg g = g_cur;
+      const int n = g.t_hi - g.t_lo;
       for (int i = 0; i < n && ok; ++i) {
         // ---- send: read page tg's partial score, pass it to the peer ----
         const uint32_t xb = tg % XBUF;
@@ -507,28 +565,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_before();
         mbar_arrive(s_free);
         {
-          const uint32_t dst = peer_x + xb * X_BYTES + r * 128 + h * 64;
-          const uint32_t pbar = peer_xbar + xb * 8;
+          // Stage this warp's 32 rows (2 KB) and ship them with one bulk
+          // copy.  The previous copy from the staging block went out a page
+          // ago; its source must have been read before it is overwritten.
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            st_async_peer_v4(dst + u * 16, make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]),
-                             pbar);
+            *reinterpret_cast<uint4*>(sXS + x_off(r, h, u)) =
+                make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]);
+          fence_proxy_async_smem();  // the copy engine reads what the threads wrote
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t blk = (uint32_t)(h * (X_BYTES / 2) + (warp & 3) * 2048);
+            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, 2048, peer_xbar + xb * 8);
+            bulk_commit();
+          }
         }
         if (h == 0 && r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
         // The segment's scores are all read after its last page, so the next
         // segment's Q may replace this one's.
-        if (i + 1 == n && si + 1 < seg_hi) load_q(segs[si + 1].rb);
+        if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
         // ---- finish the previous page ----
-        if (fin_si >= 0 && !(ok = finish(fin_si, fin_i, fin_tg, own))) break;
+        if (fin_any && !(ok = finish(fin_g, fin_i, fin_tg, own))) break;
 #pragma unroll
         for (int j = 0; j < 16; ++j) own[j] = cur[j];
-        fin_si = si;
+        fin_g = g;
+        fin_any = true;
         fin_i = i;
         fin_tg = tg;
         ++tg;
       }
+      g_cur = g_nxt;
+      if (si + 2 < seg_hi) g_nxt = segs[si + 2];
     }
-    if (ok && fin_si >= 0) ok = finish(fin_si, fin_i, fin_tg, own);
+    if (ok && fin_any) ok = finish(fin_g, fin_i, fin_tg, own);
+    if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
   }
 
   tc_fence_before();

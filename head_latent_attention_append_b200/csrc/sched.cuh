@@ -19,11 +19,15 @@
 
 namespace mla {
 
-struct Seg {
+// 32 bytes, read with two vector loads: a worker needs everything about a
+// segment (its row block's key count too) from one round trip to memory.
+struct __align__(16) Seg {
   int rb;      // row block
   int t_lo;    // first tile (inclusive), relative to the row block
   int t_hi;    // last tile (exclusive)
   int slot;    // partial slot, or -1 when the segment covers the whole row block
+  int nkeys;   // keys of the row block (its causal length)
+  int pad[3];
 };
 
 struct Sched {
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
       g.t_lo = a0;
       g.t_hi = a1;
       g.slot = whole ? -1 : (rb == r0 ? 2 * w : 2 * w + 1);
+      g.nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
+      g.pad[0] = g.pad[1] = g.pad[2] = 0;
       a.s.segs[s] = g;
       if (a0 == 0) a.s.rb_seg_first[rb] = s;
     }

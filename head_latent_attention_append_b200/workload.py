@@ -54,8 +54,9 @@ class Setup:
         return int(self.kv_len_host.max())
 
     def cache_bytes_read(self) -> int:
-        """Latent-cache bytes one step's attention must read: every key of
-        every query token's row block once (the algorithmic count)."""
+        """Latent-cache bytes the attention kernel streams: every key of every
+        query token's row block once (each query token is its own row block,
+        so a sequence with n_q new tokens is read n_q times)."""
         wl = self.wl
         esz = 2 if wl.dtype == "bf16" else 4
         if wl.mode == "prefill":
@@ -63,6 +64,15 @@ class Setup:
             keys = wl.B * S * (S + 1) // 2
         else:
             keys = int(sum(int(L) - wl.n_q + 1 + q for L in self.kv_len_host for q in range(wl.n_q)))
+        return keys * wl.d_cr * esz
+
+    def cache_bytes_unique(self) -> int:
+        """Latent-cache bytes of every sequence's history, counted once: the
+        least a step's attention must read, however many query tokens a
+        sequence brings."""
+        wl = self.wl
+        esz = 2 if wl.dtype == "bf16" else 4
+        keys = wl.B * wl.n_q if wl.mode == "prefill" else int(self.kv_len_host.sum())
         return keys * wl.d_cr * esz
 
     def attention_flops(self) -> int:
