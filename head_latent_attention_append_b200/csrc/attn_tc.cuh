@@ -26,20 +26,29 @@
 // the same two numbers, so both see bit-identical scores and run identical
 // softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
 // half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
-// P [480, 512).  Shared memory: a 3-deep ring of per-page column groups
-// (<= 5 chunks of 64 keys x 64 columns, 128-byte swizzle, loaded by TMA) and
-// five 16 KB exchange buffers, filled by the peer with bulk copies (one per
-// softmax warp per page, staged in a local 16 KB block) that complete on this
-// CTA's mbarrier; there are enough buffers that the pipeline itself keeps the
-// peer from overwriting an unread one (see XBUF).
-// The softmax runs one page behind the score MMA so the exchange round trip
-// overlaps the next page.
+// P [480, 512).
 //
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = score-MMA issuer,
-// warp 3 = P*V-MMA issuer (all warp-uniform; one elected lane issues), warp 2 =
-// TMEM allocator, warps 4-11 = two softmax / exchange / epilogue warpgroups
-// (each owns half of the keys of every row; thread r owns row r = TMEM lane
-// r).  Every wait is bounded (sm100::mbar_wait).
+// Shared memory (128-byte swizzled 64 x 64 chunks, loaded by TMA):
+//   score ring, 2 slots: this CTA's columns of a page (<= 5 chunks), freed as
+//     soon as the page's score MMA completes;
+//   latent ring, 2 slots: the page's latent columns again (4 chunks) for
+//     P*V, freed by P*V.  The second read is an L2 hit (the first was a few
+//     microseconds earlier), so HBM still sees every byte once; decoupling
+//     the rings keeps a page's HBM load off the softmax's critical loop;
+//   four 16 KB exchange buffers, filled by the peer with bulk copies (one
+//     2 KB copy per softmax warp per page, staged in a local 16 KB block) that
+//     complete on this CTA's mbarrier; four buffers make an overwrite of an
+//     unread one impossible (see XBUF).
+// The softmax runs one page behind the score MMA so the exchange overlaps the
+// next page.  Segment metadata and page ids are loaded a step ahead so no
+// global load sits on a page's critical path.
+//
+// Warp roles (384 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
+// allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
+// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-11 =
+// two softmax / exchange / epilogue warpgroups (each owns half of the keys of
+// every row; thread r owns row r = TMEM lane r).  Every wait is bounded
+// (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -51,30 +60,40 @@ using namespace sm100;
 constexpr int THREADS = 384;
 constexpr int KT = 64;                        // keys per tile (one page)
 constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
-constexpr int MAX_OWN = 5;                    // chunks per CTA per page
-constexpr int GROUPS = 3;                     // page groups in flight
-constexpr int XBUF = 5;                       // exchange buffers per CTA
-// A CTA refills the peer's exchange buffer for page t + XBUF only after its
-// own page group of page t + XBUF - GROUPS has been consumed by P*V, which
-// needs the peer's partial of that page, which the peer sends after reading
-// page t's buffer whenever t + XBUF - GROUPS >= t + 2 (the softmax runs one
-// page behind).  So no partial can overwrite one that is still unread, with
-// no extra barrier.
-static_assert(XBUF >= GROUPS + 2, "exchange buffers must outlast the page ring by the softmax lag + 1");
-constexpr int GROUP_BYTES = MAX_OWN * CHUNK_BYTES;
+constexpr int MAX_OWN = 5;                    // score chunks per CTA per page
+constexpr int MAX_PV = 4;                     // latent chunks per CTA per page (d_c <= 512)
+constexpr int SGROUPS = 2;                    // score ring: a page's own columns, freed by its score MMA
+constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
+constexpr int XBUF = 4;                       // exchange buffers per CTA
+// A CTA reads the peer's partial of page t (finish of page t) before it sends
+// its own partial of page t + 2 (the softmax runs one page behind), and the
+// peer refills that buffer with page t + XBUF only after its own finish of
+// page t + 2, which waits for that send.  Within an iteration a CTA sends page
+// k and then finishes page k - 1, so with XBUF >= 4 the refill (page t + 4,
+// iteration t + 4) always follows the finish of page t + 2 (iteration t + 3):
+// no partial can overwrite one that is still unread, with no extra barrier.
+static_assert(XBUF >= 4, "the exchange needs softmax lag (1) * 2 + 2 buffers");
+constexpr int SG_BYTES = MAX_OWN * CHUNK_BYTES;
+constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
 
-constexpr int OFF_G = 0;
-constexpr int OFF_X = OFF_G + GROUPS * GROUP_BYTES;
+// The exchange buffers and their barriers sit at the same offsets in both
+// CTAs (the peer addresses them through mapa).
+constexpr int OFF_X = 0;
 constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
-constexpr int OFF_MH = OFF_XS + X_BYTES;          // half-row maxima [2][2][128] fp32
-constexpr int OFF_LS = OFF_MH + 2 * 2 * 128 * 4;  // half-row sums [2][128] fp32
-constexpr int OFF_BAR = OFF_LS + 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * GROUPS + XBUF + 7 + 4;
+constexpr int OFF_SG = OFF_XS + X_BYTES;
+constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
+constexpr int OFF_MH = OFF_VG + VGROUPS * VG_BYTES;  // half-row maxima [2][2][128] fp32 (sums reuse a slot)
+constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
+constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 7 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to 1024
+// No slack for aligning the base: the kernel has no static shared memory, so
+// its dynamic block starts on a 1024-byte boundary (the kernel checks this
+// and reports MLA_ERR_UNSUPPORTED otherwise).
+constexpr size_t SMEM_BYTES = SMEM_USED;
+static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA can have");
 
 struct Params {
   AttnArgs a;
@@ -147,13 +166,18 @@ __device__ __forceinline__ uint32_t x_off(int r, int h, int u) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
+    if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* g_full = bars;
-  uint64_t* g_empty = bars + GROUPS;
-  uint64_t* x_full = bars + 2 * GROUPS;  // [XBUF] the peer's partial has landed here
-  uint64_t* s_full = x_full + XBUF;
+  uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
+  uint64_t* sg_full = x_full + XBUF;     // [SGROUPS]
+  uint64_t* sg_empty = sg_full + SGROUPS;
+  uint64_t* vg_full = sg_empty + SGROUPS;  // [VGROUPS]
+  uint64_t* vg_empty = vg_full + VGROUPS;
+  uint64_t* s_full = vg_empty + VGROUPS;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_full + 2;
   uint64_t* pv_done = s_full + 3;
@@ -175,9 +199,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
   if (tid == 32) {
-    for (int i = 0; i < GROUPS; ++i) {
-      mbar_init(&g_full[i], 1);
-      mbar_init(&g_empty[i], 1);
+    for (int i = 0; i < SGROUPS; ++i) {
+      mbar_init(&sg_full[i], 1);
+      mbar_init(&sg_empty[i], 1);
+    }
+    for (int i = 0; i < VGROUPS; ++i) {
+      mbar_init(&vg_full[i], 1);
+      mbar_init(&vg_empty[i], 1);
     }
     for (int i = 0; i < XBUF; ++i) mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
     mbar_init(s_full, 1);
@@ -202,10 +230,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 2) {
+    // ---------------------------------------------------- TMA producers
+    // Warp 0 fills the score ring with this CTA's columns of each page;
+    // warp 2 fills the latent ring with the page's latent columns again
+    // (an L2 hit: the score ring read them a few microseconds earlier).
     // Metadata loads run one step ahead: the next segment while this one
     // streams, the next page id while this page waits for its ring slot.
+    const bool score_ring = warp == 0;
+    const int nring = score_ring ? SGROUPS : VGROUPS;
+    const int nchunk = score_ring ? n_own : npv;
+    const int ring_bytes = score_ring ? SG_BYTES : VG_BYTES;
+    uint8_t* ring = smem + (score_ring ? OFF_SG : OFF_VG);
+    uint64_t* full = score_ring ? sg_full : vg_full;
+    uint64_t* empty = score_ring ? sg_empty : vg_empty;
     uint32_t cnt = 0;
     if (seg_lo < seg_hi) {
       int si = seg_lo;
@@ -226,17 +264,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         if (more) page_n = a.page_table[(long long)(g.rb / a.n_q) * a.max_pages + t];
-        const uint32_t gs = cnt % GROUPS;
-        if (!mbar_wait_warp(&g_empty[gs], ((cnt / GROUPS) & 1) ^ 1, abort_flag, a.err)) break;
+        const uint32_t gs = cnt % nring;
+        if (!mbar_wait_warp(&empty[gs], ((cnt / nring) & 1) ^ 1, abort_flag, a.err)) break;
         if (page < 0 || page >= a.num_pages) {
-          if (rank == 0 && elect_one()) flag_error(a.err, kErrBounds);
+          if (rank == 0 && score_ring && elect_one()) flag_error(a.err, kErrBounds);
           page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(&g_full[gs], n_own * CHUNK_BYTES);
-          for (int q = 0; q < n_own; ++q)
-            tma_load_2d(smem + OFF_G + gs * GROUP_BYTES + q * CHUNK_BYTES, &tmap, (c_lo + q) * 64, page * KT,
-                        &g_full[gs]);
+          mbar_arrive_expect_tx(&full[gs], nchunk * CHUNK_BYTES);
+          for (int q = 0; q < nchunk; ++q)
+            tma_load_2d(ring + gs * ring_bytes + q * CHUNK_BYTES, &tmap, (c_lo + q) * 64, page * KT, &full[gs]);
         }
         __syncwarp();
         ++cnt;
@@ -244,9 +281,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     if (*abort_flag) {
       // Let every copy already issued land before the CTA can exit.
-      for (uint32_t q = 0; q < GROUPS && q < cnt; ++q) {
-        const uint32_t last = q + GROUPS * ((cnt - 1 - q) / GROUPS);
-        mbar_wait_warp(&g_full[q], (last / GROUPS) & 1, abort_flag, nullptr, 50000000ull, false);
+      for (uint32_t q = 0; q < (uint32_t)nring && q < cnt; ++q) {
+        const uint32_t last = q + nring * ((cnt - 1 - q) / nring);
+        mbar_wait_warp(&full[q], (last / nring) & 1, abort_flag, nullptr, 50000000ull, false);
       }
     }
   } else if (warp == 1 || warp == 3) {
@@ -255,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // only on its own inputs, and each tcgen05.commit tracks only the MMAs
     // its own thread issued.
     const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q, tP = tbase + TM_P;
-    const uint32_t sG = smem_u32(smem + OFF_G);
+    const uint32_t sSG = smem_u32(smem + OFF_SG), sVG = smem_u32(smem + OFF_VG);
     uint32_t tg = 0, seg_k = 0;
     bool ok = true;
     if (warp == 1) {
@@ -269,11 +306,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_after();
         for (int i = 0; i < n; ++i) {
           if (tg > 0 && !(ok = mbar_wait_warp(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
-          const uint32_t gs = tg % GROUPS;
-          if (!(ok = mbar_wait_warp(&g_full[gs], (tg / GROUPS) & 1, abort_flag, a.err))) break;
+          const uint32_t gs = tg % SGROUPS;
+          if (!(ok = mbar_wait_warp(&sg_full[gs], (tg / SGROUPS) & 1, abort_flag, a.err))) break;
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t gb = sG + gs * GROUP_BYTES;
+            const uint32_t gb = sSG + gs * SG_BYTES;
             for (int q = 0; q < n_own; ++q) {
 #pragma unroll
               for (int k = 0; k < 4; ++k)
@@ -281,6 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                        (q | k) ? 1u : 0u);
             }
             tc_commit(s_full);
+            tc_commit(&sg_empty[gs]);  // the score ring slot is free once its MMAs are done
           }
           __syncwarp();
           ++tg;
@@ -297,15 +335,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int i = 0; i < n; ++i) {
           if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
           if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
+          const uint32_t vs = tg % VGROUPS;
+          if (!(ok = mbar_wait_warp(&vg_full[vs], (tg / VGROUPS) & 1, abort_flag, a.err))) break;
           tc_fence_after();
-          const uint32_t gs = tg % GROUPS;
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < KT / 16; ++kk)
-              mma_ts(tO, tP + kk * 8, sdesc_sw128(sG + gs * GROUP_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
+              mma_ts(tO, tP + kk * 8, sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
                      (i == 0 && kk == 0) ? 0u : 1u);
             tc_commit(pv_done);
-            tc_commit(&g_empty[gs]);
+            tc_commit(&vg_empty[vs]);
           }
           __syncwarp();
           ++tg;
@@ -332,12 +371,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P + 16 * h;
     uint64_t* pair_bar = &pair_bars[warp & 3];
     uint32_t pair_phase = 0;
-    uint8_t* sG = smem + OFF_G;
+    uint8_t* sV = smem + OFF_VG;
     uint8_t* sX = smem + OFF_X;
     uint8_t* sXS = smem + OFF_XS;
     const int lane = tid & 31;
     float* mh = reinterpret_cast<float*>(smem + OFF_MH);
-    float* ls = reinterpret_cast<float*>(smem + OFF_LS);
     const uint32_t peer_x = map_peer(smem_u32(sX), peer);
     const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
     const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
@@ -475,8 +513,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       l += psum;
       if (valid_all < KT) {
         // Keys past the end: P is 0 there, but 0 * NaN would still poison O,
-        // so clear those rows of this tile's latent chunks.
-        uint8_t* gb = sG + (tgf % GROUPS) * GROUP_BYTES;
+        // so clear those rows of this tile's latent chunks (once they landed).
+        if (!wait_all(&vg_full[tgf % VGROUPS], (tgf / VGROUPS) & 1)) return false;
+        uint8_t* gb = sV + (tgf % VGROUPS) * VG_BYTES;
         const int rows = KT - valid_all, units = rows * 8 * npv;
         for (int x = r + 128 * h; x < units; x += 256) {
           const int q = x / (rows * 8), rem = x - q * rows * 8;
@@ -492,7 +531,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // ---- epilogue of the segment ----
       if (!wait_all(pv_done, tgf & 1)) return false;
       tc_fence_after();
-      // Row sum: both halves add the two partial sums in the same order.
+      // Row sum: both halves add the two partial sums in the same order.  The
+      // sums borrow the max slot of the previous page: the partner read that
+      // page's maxima before the last pair sync, and the next page's maxima
+      // go there only after the second sync below.
+      float* ls = mh + ((tgf + 1) & 1) * 256;
       ls[h * 128 + r] = l;
       if (!pair_sync()) return false;
       const float lrow = ls[r] + ls[128 + r];
