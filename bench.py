@@ -119,6 +119,25 @@ def barrier(ws):
         dist.barrier()
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    capture (profiles/traffic.json), or None when there is none for this
+    workload or the kernel's sources changed since it was taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        rec = json.load(fh).get(workload)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in rec["source_files"]:
+        with open(os.path.join(ROOT, "head_latent_attention_append_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return rec["traffic_bytes"] if h.hexdigest() == rec["source_sha256"] else None
+
+
 PREFILL_SAMPLE_TOKENS = 1024   # causal prefix of one sequence per oracle prefill sample
 
 
@@ -323,7 +342,8 @@ def run_ours(args):
                "frac": tc_tflops / tc_peak, "algorithmic_flops_per_launch": flops,
                "peak_kind": "bf16 sustained"}
     main_roof, other_roof = (tc_roof, hbm_roof) if prefill else (hbm_roof, tc_roof)
-    roofline = dict(main_roof, traffic=None, kernel="latent attention (split-KV)", peak_src=peaks["src"],
+    roofline = dict(main_roof, traffic=measured_traffic(wl.name), kernel="latent attention (split-KV)",
+                    peak_src=peaks["src"],
                     avg_kernel_ms=attn_avg_ms, streamed_cache_bytes_per_launch=streamed_bytes,
                     other_roof=other_roof)
     l2_note = (f"inputs larger than L2: {wl.B * wl.n_q * wl.d_model * 2 / 1e6:.0f} MB of hidden states in and "

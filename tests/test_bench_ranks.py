@@ -53,3 +53,23 @@ def test_single_rank_is_passthrough():
     import bench
     ms, value = bench.aggregate(604_053_504, 0.5, 1)
     assert ms == 0.5 and value == pytest.approx(604_053_504 / 0.5e-3 / 1e9)
+
+
+def test_measured_traffic_follows_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from a recorded ncu capture only while the
+    kernel sources still hash to what was captured."""
+    import hashlib
+    import json
+    import bench
+    csrc = tmp_path / "head_latent_attention_append_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cuh").write_bytes(b"kernel v1")
+    digest = hashlib.sha256(b"kernel v1").hexdigest()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"wl": {"traffic_bytes": 1234, "source_files": ["k.cuh"], "source_sha256": digest}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("wl") == 1234
+    assert bench.measured_traffic("other") is None
+    (csrc / "k.cuh").write_bytes(b"kernel v2")
+    assert bench.measured_traffic("wl") is None
