@@ -36,19 +36,20 @@
 //     microseconds earlier), so HBM still sees every byte once; decoupling
 //     the rings keeps a page's HBM load off the softmax's critical loop;
 //   four 16 KB exchange buffers, filled by the peer with bulk copies (one
-//     2 KB copy per softmax warp per page, staged in a local 16 KB block) that
+//     4 KB copy per sender warp per page, staged in a local 16 KB block) that
 //     complete on this CTA's mbarrier; four buffers make an overwrite of an
 //     unread one impossible (see XBUF).
-// The softmax runs one page behind the score MMA so the exchange overlaps the
-// next page.  Segment metadata and page ids are loaded a step ahead so no
-// global load sits on a page's critical path.
+// Segment metadata and page ids are loaded a step ahead so no global load
+// sits on a page's critical path.
 //
 // Warp roles (384 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
 // allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
-// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-11 =
-// two softmax / exchange / epilogue warpgroups (each owns half of the keys of
-// every row; thread r owns row r = TMEM lane r).  Every wait is bounded
-// (sm100::mbar_wait).
+// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-7 =
+// sender (reads each page's partial score, ships it to the peer, loads Q),
+// warps 8-11 = finisher (whole rows: combine, softmax, P, epilogue); thread r
+// of either owns row r = TMEM lane r.  The sender runs a page ahead of the
+// finisher, so the exchange of one page overlaps the softmax of the previous
+// one.  Every wait is bounded (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -65,14 +66,13 @@ constexpr int MAX_PV = 4;                     // latent chunks per CTA per page 
 constexpr int SGROUPS = 2;                    // score ring: a page's own columns, freed by its score MMA
 constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
 constexpr int XBUF = 4;                       // exchange buffers per CTA
-// A CTA reads the peer's partial of page t (finish of page t) before it sends
-// its own partial of page t + 2 (the softmax runs one page behind), and the
-// peer refills that buffer with page t + XBUF only after its own finish of
-// page t + 2, which waits for that send.  Within an iteration a CTA sends page
-// k and then finishes page k - 1, so with XBUF >= 4 the refill (page t + 4,
-// iteration t + 4) always follows the finish of page t + 2 (iteration t + 3):
-// no partial can overwrite one that is still unread, with no extra barrier.
-static_assert(XBUF >= 4, "the exchange needs softmax lag (1) * 2 + 2 buffers");
+// No partial can overwrite one that is still unread, with no extra barrier:
+// a CTA's finisher reads the peer's partial of page t before it takes its own
+// page t + 1 out of the staging block, which the sender needs before it ships
+// page t + 2.  The peer's finisher waits for that page t + 2 before it takes
+// its own page t + 3 out of staging, which the peer's sender needs before it
+// ships page t + 4 into the buffer page t used.
+static_assert(XBUF >= 4, "the exchange needs four buffers (see above)");
 constexpr int SG_BYTES = MAX_OWN * CHUNK_BYTES;
 constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
@@ -84,15 +84,11 @@ constexpr int OFF_X = 0;
 constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
 constexpr int OFF_SG = OFF_XS + X_BYTES;
 constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
-constexpr int OFF_MH = OFF_VG + VGROUPS * VG_BYTES;  // half-row maxima [2][2][128] fp32 (sums reuse a slot)
-constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 7 + 4;
+constexpr int OFF_BAR = OFF_VG + VGROUPS * VG_BYTES;
+constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 9;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-// No slack for aligning the base: the kernel has no static shared memory, so
-// its dynamic block starts on a 1024-byte boundary (the kernel checks this
-// and reports MLA_ERR_UNSUPPORTED otherwise).
-constexpr size_t SMEM_BYTES = SMEM_USED;
+constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to 1024
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA can have");
 
 struct Params {
@@ -155,22 +151,18 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// Byte offset, in an exchange tile, of 16-byte piece u (0..3) of the 32
-// partial scores that thread r of warpgroup h owns.  Layout [h][r][64 bytes],
-// so each warp's 32 rows form one contiguous 2 KB block (one bulk copy); the
-// pieces are XOR-swizzled by (r >> 1) so that the eight rows a quarter-warp
-// touches at once fall in eight different bank groups.
-__device__ __forceinline__ uint32_t x_off(int r, int h, int u) {
-  return (uint32_t)(h * (X_BYTES / 2) + r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
-}
+// Byte offset, in an exchange tile, of 16-byte piece u (0..7) of row r's 64
+// bf16 partial scores.  Layout [row][128 bytes], so each warp's 32 rows form
+// one contiguous 4 KB block (one bulk copy); the pieces are XOR-swizzled by
+// the row so that the eight rows a quarter-warp touches at once fall in
+// eight different bank groups.
+constexpr int X_WARP_BYTES = 32 * KT * 2;
+__device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
-    if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
-    return;
-  }
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
   uint64_t* sg_full = x_full + XBUF;     // [SGROUPS]
@@ -184,7 +176,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* q_ready = s_full + 4;
   uint64_t* o_free = s_full + 5;
   uint64_t* final_bar = s_full + 6;
-  uint64_t* pair_bars = s_full + 7;  // [4]: the two softmax warps of a lane quarter
+  uint64_t* xs_full = s_full + 7;  // the sender has staged a page's partial
+  uint64_t* xs_free = s_full + 8;  // the finisher has taken it out of the staging block
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -209,13 +202,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < XBUF; ++i) mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
     mbar_init(s_full, 1);
-    mbar_init(s_free, 256);
-    mbar_init(p_ready, 256);
+    mbar_init(s_free, 128);   // sender
+    mbar_init(p_ready, 128);  // finisher
     mbar_init(pv_done, 1);
-    mbar_init(q_ready, 256);
-    mbar_init(o_free, 256);
+    mbar_init(q_ready, 128);  // sender
+    mbar_init(o_free, 128);   // finisher
     mbar_init(final_bar, 2);  // one commit per issuer warp
-    for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
+    mbar_init(xs_full, 128);
+    mbar_init(xs_free, 128);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -356,294 +350,275 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     __syncwarp();
     mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
   } else if (warp >= 4) {
-    // ------------------------------- softmax, score exchange and epilogue
-    // Two warpgroups: WG h (warps 4+4h .. 7+4h) owns keys [32h, 32h + 32) of
-    // every row; thread r of a WG owns row r (= TMEM lane r).  The two threads
-    // of a row agree on the row maximum through a 64-arrival mbarrier (their
-    // warps share a lane quarter).  The softmax runs one page behind the
-    // score: "send" reads page t's partial score and passes it to the peer,
-    // then "finish" completes page t-1, whose peer half has had a page's time
-    // to arrive.
-    const int h = warp >= 8 ? 1 : 0;
-    const int r = tid - 128 - 128 * h;
+    // ------------------------------------------- sender and finisher warpgroups
+    // Thread r of either warpgroup owns row r (= TMEM lane r) of the page.
+    // The sender (warps 4-7) reads each page's partial score (all 64 keys),
+    // packs it to bf16, stages it and ships it to the peer with one bulk copy
+    // per warp; it also loads each segment's Q slice.  The finisher (warps
+    // 8-11) owns whole rows: it adds its own staged partial to the peer's,
+    // keeps the running max and sum, writes P and runs the segment epilogue.
+    // The two work on consecutive pages at once, so the exchange of page t+1
+    // overlaps the softmax of page t, and no row is split between threads.
+    const bool sender = warp < 8;
+    const int r = tid - (sender ? 128 : 256);
+    const int lane = tid & 31;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tbase + lane_off + TM_S + 32 * h, tO = tbase + lane_off + TM_O;
-    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P + 16 * h;
-    uint64_t* pair_bar = &pair_bars[warp & 3];
-    uint32_t pair_phase = 0;
-    uint8_t* sV = smem + OFF_VG;
+    const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O;
+    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P;
     uint8_t* sX = smem + OFF_X;
     uint8_t* sXS = smem + OFF_XS;
-    const int lane = tid & 31;
-    float* mh = reinterpret_cast<float*>(smem + OFF_MH);
-    const uint32_t peer_x = map_peer(smem_u32(sX), peer);
-    const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
-    const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
-    const int hc0 = h * (dh / 64), hc1 = hc0 + dh / 64;  // this WG's 32-column chunks of O
     bool ok = true;
-
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
       return __all_sync(0xffffffffu, r_ok);
     };
-    // Meeting point of the two threads of a row (bounded, like every wait).
-    auto pair_sync = [&]() -> bool {
-      mbar_arrive(pair_bar);
-      bool r_ok = mbar_wait(pair_bar, pair_phase & 1, abort_flag, a.err);
-      ++pair_phase;
-      return __all_sync(0xffffffffu, r_ok);
-    };
-    // Row r of this CTA's Q slice (chunks c_lo .. c_lo + n_own - 1) into TMEM;
-    // the two warpgroups take alternate chunks.
-    auto load_q = [&](int rb) {
-      const uint4* src =
-          (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
-      for (int q = h; q < n_own; q += 2) {
-        uint32_t wv[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int col = (c_lo + q) * 64 + u * 8;
-          uint4 v = (src && col < a.d_cr) ? __ldg(src + col / 8) : make_uint4(0, 0, 0, 0);
-          wv[4 * u + 0] = v.x;
-          wv[4 * u + 1] = v.y;
-          wv[4 * u + 2] = v.z;
-          wv[4 * u + 3] = v.w;
-        }
-        tmem_st32(tQ + q * 32, wv);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(q_ready);
-    };
 
-    float m_used = -INFINITY, l = 0.f;
-    // Finish tile i of segment g (global tile tgf): combine the two bf16
-    // partial scores, softmax, P into TMEM; the segment's epilogue after its
-    // last tile.
-    auto finish = [&](const Seg& g, int i, uint32_t tgf, const uint32_t (&mine)[16]) -> bool {
-      const int rb = g.rb;
-      const int t = g.t_lo + i;
-      const int nkeys = g.nkeys;
-      const uint32_t xb = tgf % XBUF;
-      if (!__all_sync(0xffffffffu, mbar_wait(&x_full[xb], (tgf / XBUF) & 1, abort_flag, a.err, 2000000000ull, true,
-                                             true)))
-        return false;
-      float s[32];
-      {
-        const uint8_t* src = sX + xb * X_BYTES;
+    if (sender) {
+      const uint32_t peer_x = map_peer(smem_u32(sX), peer);
+      const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
+      const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
+      // Row r of this CTA's Q slice (chunks c_lo .. c_lo + n_own - 1) into TMEM.
+      auto load_q = [&](int rb) {
+        const uint4* src =
+            (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
+        for (int q = 0; q < n_own; ++q) {
+          uint32_t wv[32];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, h, u));
-          const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_bf16x2(mine[4 * u + e]);
-            const float2 y = unpack_bf16x2(pw[e]);
-            s[8 * u + 2 * e] = x.x + y.x;
-            s[8 * u + 2 * e + 1] = x.y + y.y;
+          for (int u = 0; u < 8; ++u) {
+            const int col = (c_lo + q) * 64 + u * 8;
+            uint4 v = (src && col < a.d_cr) ? __ldg(src + col / 8) : make_uint4(0, 0, 0, 0);
+            wv[4 * u + 0] = v.x;
+            wv[4 * u + 1] = v.y;
+            wv[4 * u + 2] = v.z;
+            wv[4 * u + 3] = v.w;
           }
+          tmem_st32(tQ + q * 32, wv);
         }
-      }
-      const int valid_all = min(KT, nkeys - t * KT);
-      const int valid = valid_all - 32 * h;  // valid keys among this WG's 32
-      if (valid < 32) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j >= valid) s[j] = -INFINITY;
-      }
-      float mt;
-      {
-        float mx[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
-#pragma unroll
-        for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-          for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-        float* slot = mh + (tgf & 1) * 256;
-        slot[h * 128 + r] = mx[0];
-        if (!pair_sync()) return false;
-        mt = fmaxf(slot[r], slot[128 + r]);
-      }
-      // Running max with lazy rescaling: O and l stay relative to m_used
-      // until a tile's max exceeds it by more than 2^8.
-      bool resc = false;
-      float scale = 1.f;
-      if (i == 0) {
-        m_used = mt;
-        l = 0.f;
-      } else if (mt > m_used + 8.f) {
-        scale = fast_exp2(m_used - mt);
-        m_used = mt;
-        resc = true;
-      }
-      uint32_t pk[16];
-      float psum;
-      {
-        float ps[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          ps[u] = 0.f;
-          pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u]);
-        }
-#pragma unroll
-        for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-          for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
-        psum = ps[0];
-      }
-      // The previous P*V must be done before P is overwritten or O rescaled.
-      if (tgf > 0) {
-        if (!wait_all(pv_done, (tgf - 1) & 1)) return false;
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        for (int cc = hc0; cc < hc1; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tO + cc * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
-          tmem_st32(tO + cc * 32, v);
-        }
-        l *= scale;
-      }
-      tmem_st16(tP, pk);
-      tmem_st_wait();
-      l += psum;
-      if (valid_all < KT) {
-        // Keys past the end: P is 0 there, but 0 * NaN would still poison O,
-        // so clear those rows of this tile's latent chunks (once they landed).
-        if (!wait_all(&vg_full[tgf % VGROUPS], (tgf / VGROUPS) & 1)) return false;
-        uint8_t* gb = sV + (tgf % VGROUPS) * VG_BYTES;
-        const int rows = KT - valid_all, units = rows * 8 * npv;
-        for (int x = r + 128 * h; x < units; x += 256) {
-          const int q = x / (rows * 8), rem = x - q * rows * 8;
-          *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
-              make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      mbar_arrive(p_ready);
-      if (i + 1 < g.t_hi - g.t_lo) return true;
-
-      // ---- epilogue of the segment ----
-      if (!wait_all(pv_done, tgf & 1)) return false;
-      tc_fence_after();
-      // Row sum: both halves add the two partial sums in the same order.  The
-      // sums borrow the max slot of the previous page: the partner read that
-      // page's maxima before the last pair sync, and the next page's maxima
-      // go there only after the second sync below.
-      float* ls = mh + ((tgf + 1) & 1) * 256;
-      ls[h * 128 + r] = l;
-      if (!pair_sync()) return false;
-      const float lrow = ls[r] + ls[128 + r];
-      if (!pair_sync()) return false;  // both have read before the next write
-      // A whole row block is normalised into obar (bf16); a piece of a split
-      // row block leaves its unnormalised sum and (m, l) in its slot.
-      const bool whole = g.slot < 0;
-      const float inv = 1.f / lrow;
-      for (int cc = hc0; cc < hc1; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tO + cc * 32, v);
-        tmem_ld_wait();
-        if (r < a.n_h) {
-          const int col = (int)rank * dh + cc * 32;
-          if (whole) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.obar) +
-                                                  ((long long)rb * a.n_h + r) * a.d_c + col);
-            float dummy = 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv, dummy);
-              o.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv, dummy);
-              o.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv, dummy);
-              o.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv, dummy);
-              dst[q] = o;
-            }
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(a.part_o + ((long long)g.slot * a.n_h + r) * a.d_c + col);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-        }
-      }
-      if (!whole && rank == 0 && h == 0 && r < a.n_h) {
-        a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 0] = m_used;
-        a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = lrow;
-      }
-      tc_fence_before();
-      mbar_arrive(o_free);
-      return true;
-    };
-
-    // Segment metadata stays in registers, the next segment's loaded a
-    // segment ahead, so no global load sits on a page's critical path.
-    Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-    Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
-    if (seg_lo < seg_hi) load_q(g_cur.rb);
-    uint32_t own[16];
-    Seg fin_g{};
-    bool fin_any = false;
-    int fin_i = 0;
-    uint32_t fin_tg = 0, tg = 0;
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const Seg g = g_cur;
-      const int n = g.t_hi - g.t_lo;
-      for (int i = 0; i < n && ok; ++i) {
-        // ---- send: read page tg's partial score, pass it to the peer ----
-        const uint32_t xb = tg % XBUF;
-        if (!(ok = wait_all(s_full, tg & 1))) break;
-        tc_fence_after();
-        uint32_t cur[16];
-        {
-          uint32_t v[32];
-          tmem_ld32(tS, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) cur[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-        }
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(s_free);
-        {
-          // Stage this warp's 32 rows (2 KB) and ship them with one bulk
-          // copy.  The previous copy from the staging block went out a page
-          // ago; its source must have been read before it is overwritten.
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
+        mbar_arrive(q_ready);
+      };
+      // Segment metadata stays in registers, the next segment's loaded a
+      // segment ahead.
+      Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : Seg{};
+      int n_cur = 0;
+      if (seg_lo < seg_hi) {
+        const Seg g0 = segs[seg_lo];
+        load_q(g0.rb);
+        n_cur = g0.t_hi - g0.t_lo;
+      }
+      uint32_t tg = 0;
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
+        const int n = n_cur;
+        for (int i = 0; i < n; ++i, ++tg) {
+          const uint32_t xb = tg % XBUF;
+          if (!(ok = wait_all(s_full, tg & 1))) break;
+          tc_fence_after();
+          uint32_t cur[32];
+          {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tS, v0);
+            tmem_ld32(tS + 32, v1);
+            tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(sXS + x_off(r, h, u)) =
+            for (int j = 0; j < 16; ++j) {
+              cur[j] = pack_bf16x2(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1]));
+              cur[16 + j] = pack_bf16x2(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1]));
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(s_free);
+          // The staging block is reused: the finisher must have taken the
+          // previous page out of it, and the copy engine must have read it.
+          if (lane == 0) bulk_wait_read_all();
+          if (tg > 0 && !(ok = wait_all(xs_free, (tg - 1) & 1))) break;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(sXS + x_off(r, u)) =
                 make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]);
           fence_proxy_async_smem();  // the copy engine reads what the threads wrote
           __syncwarp();
           if (lane == 0) {
-            const uint32_t blk = (uint32_t)(h * (X_BYTES / 2) + (warp & 3) * 2048);
-            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, 2048, peer_xbar + xb * 8);
+            const uint32_t blk = (uint32_t)((warp & 3) * X_WARP_BYTES);
+            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, X_WARP_BYTES, peer_xbar + xb * 8);
             bulk_commit();
           }
+          // The peer's partial of this page will land in exchange buffer xb.
+          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
+          mbar_arrive(xs_full);
+          // The segment's scores are all read after its last page, so the next
+          // segment's Q may replace this one's.
+          if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
         }
-        if (h == 0 && r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
-        // The segment's scores are all read after its last page, so the next
-        // segment's Q may replace this one's.
-        if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
-        // ---- finish the previous page ----
-        if (fin_any && !(ok = finish(fin_g, fin_i, fin_tg, own))) break;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) own[j] = cur[j];
-        fin_g = g;
-        fin_any = true;
-        fin_i = i;
-        fin_tg = tg;
-        ++tg;
+        n_cur = g_nxt.t_hi - g_nxt.t_lo;
+        if (si + 2 < seg_hi) g_nxt = segs[si + 2];
       }
-      g_cur = g_nxt;
-      if (si + 2 < seg_hi) g_nxt = segs[si + 2];
+      if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
+    } else {
+      Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
+      Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
+      uint8_t* sV = smem + OFF_VG;
+      float m_used = -INFINITY, l = 0.f;
+      uint32_t tg = 0;
+      for (int si = seg_lo; si < seg_hi && ok; ++si) {
+        const Seg g = g_cur;
+        const int n = g.t_hi - g.t_lo;
+        for (int i = 0; i < n; ++i, ++tg) {
+          const int t = g.t_lo + i;
+          const uint32_t xb = tg % XBUF;
+          // This CTA's partial, staged by the sender; the block goes straight
+          // back to it.
+          if (!(ok = wait_all(xs_full, tg & 1))) break;
+          uint4 own4[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) own4[u] = *reinterpret_cast<const uint4*>(sXS + x_off(r, u));
+          mbar_arrive(xs_free);
+          // The peer's partial (its bytes complete this CTA's barrier).
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_full[xb], (tg / XBUF) & 1, abort_flag, a.err,
+                                                       2000000000ull, true, true))))
+            break;
+          float s[64];
+          {
+            const uint8_t* src = sX + xb * X_BYTES;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, u));
+              const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+              const uint32_t mw[4] = {own4[u].x, own4[u].y, own4[u].z, own4[u].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 x = unpack_bf16x2(mw[e]);
+                const float2 y = unpack_bf16x2(pw[e]);
+                s[8 * u + 2 * e] = x.x + y.x;
+                s[8 * u + 2 * e + 1] = x.y + y.y;
+              }
+            }
+          }
+          const int valid = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
+          if (valid < KT) {
+#pragma unroll
+            for (int j = 0; j < KT; ++j)
+              if (j >= valid) s[j] = -INFINITY;
+          }
+          float mt;
+          {
+            float mx[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mx[j] = fmaxf(s[j], s[j + 32]);
+#pragma unroll
+            for (int w2 = 16; w2 >= 1; w2 >>= 1)
+#pragma unroll
+              for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+            mt = mx[0];
+          }
+          // Running max with lazy rescaling: O and l stay relative to m_used
+          // until a page's max exceeds it by more than 2^8.
+          bool resc = false;
+          float scale = 1.f;
+          if (i == 0) {
+            m_used = mt;
+            l = 0.f;
+          } else if (mt > m_used + 8.f) {
+            scale = fast_exp2(m_used - mt);
+            m_used = mt;
+            resc = true;
+          }
+          uint32_t pk[32];
+          float psum;
+          {
+            float ps[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) ps[u] = 0.f;
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u & 15]);
+#pragma unroll
+            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+              for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
+            psum = ps[0];
+          }
+          // The previous P*V must be done before P is overwritten or O rescaled.
+          if (tg > 0) {
+            if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
+            tc_fence_after();
+          }
+          if (__any_sync(0xffffffffu, resc)) {
+            for (int cc = 0; cc < dh / 32; ++cc) {
+              uint32_t v[32];
+              tmem_ld32(tO + cc * 32, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
+              tmem_st32(tO + cc * 32, v);
+            }
+            l *= scale;
+          }
+          tmem_st32(tP, pk);
+          tmem_st_wait();
+          l += psum;
+          if (valid < KT) {
+            // Keys past the end: P is 0 there, but 0 * NaN would still poison
+            // O, so clear those rows of this page's latent chunks (once they
+            // have landed).
+            if (!(ok = wait_all(&vg_full[tg % VGROUPS], (tg / VGROUPS) & 1))) break;
+            uint8_t* gb = sV + (tg % VGROUPS) * VG_BYTES;
+            const int rows = KT - valid, units = rows * 8 * npv;
+            for (int x = r; x < units; x += 128) {
+              const int q = x / (rows * 8), rem = x - q * rows * 8;
+              *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+          tc_fence_before();
+          mbar_arrive(p_ready);
+          if (i + 1 < n) continue;
+
+          // ---- epilogue of the segment ----
+          if (!(ok = wait_all(pv_done, tg & 1))) break;
+          tc_fence_after();
+          // A whole row block is normalised into obar (bf16); a piece of a
+          // split row block leaves its unnormalised sum and (m, l) in its slot.
+          const bool whole = g.slot < 0;
+          const float inv = 1.f / l;
+          for (int cc = 0; cc < dh / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tO + cc * 32, v);
+            tmem_ld_wait();
+            if (r < a.n_h) {
+              const int col = (int)rank * dh + cc * 32;
+              if (whole) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.obar) +
+                                                      ((long long)g.rb * a.n_h + r) * a.d_c + col);
+                float dummy = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  uint4 o;
+                  o.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv, dummy);
+                  o.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv, dummy);
+                  o.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv, dummy);
+                  o.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv, dummy);
+                  dst[q] = o;
+                }
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(a.part_o + ((long long)g.slot * a.n_h + r) * a.d_c + col);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              }
+            }
+          }
+          if (!whole && rank == 0 && r < a.n_h) {
+            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 0] = m_used;
+            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = l;
+          }
+          tc_fence_before();
+          mbar_arrive(o_free);
+        }
+        g_cur = g_nxt;
+        if (si + 2 < seg_hi) g_nxt = segs[si + 2];
+      }
     }
-    if (ok && fin_any) ok = finish(fin_g, fin_i, fin_tg, own);
-    if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
   }
 
   tc_fence_before();
