@@ -42,13 +42,14 @@
 // Segment metadata and page ids are loaded a step ahead so no global load
 // sits on a page's critical path.
 //
-// Warp roles (384 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
+// Warp roles (512 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
 // allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
 // P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-7 =
 // sender (reads each page's partial score, ships it to the peer, loads Q),
-// warps 8-11 = finisher (whole rows: combine, softmax, P, epilogue); thread r
-// of either owns row r = TMEM lane r.  The sender runs a page ahead of the
-// finisher, so the exchange of one page overlaps the softmax of the previous
+// warps 8-11 and 12-15 = the two finisher halves (keys 0-31 and 32-63 of
+// every row: combine, softmax, P, and half of O in the epilogue); thread r of
+// any of these owns row r = TMEM lane r.  The sender runs a page ahead of the
+// finishers, so the exchange of one page overlaps the softmax of the previous
 // one.  Every wait is bounded (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
@@ -58,7 +59,7 @@ namespace mla {
 namespace attn_tc {
 using namespace sm100;
 
-constexpr int THREADS = 384;
+constexpr int THREADS = 512;
 constexpr int KT = 64;                        // keys per tile (one page)
 constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
 constexpr int MAX_OWN = 5;                    // score chunks per CTA per page
@@ -67,11 +68,11 @@ constexpr int SGROUPS = 2;                    // score ring: a page's own column
 constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
 constexpr int XBUF = 4;                       // exchange buffers per CTA
 // No partial can overwrite one that is still unread, with no extra barrier:
-// a CTA's finisher reads the peer's partial of page t before it takes its own
-// page t + 1 out of the staging block, which the sender needs before it ships
-// page t + 2.  The peer's finisher waits for that page t + 2 before it takes
-// its own page t + 3 out of staging, which the peer's sender needs before it
-// ships page t + 4 into the buffer page t used.
+// each finisher half reads the peer's partial of page t before it takes its
+// own page t + 1 out of the staging block, which the sender needs (from both
+// halves) before it ships page t + 2.  The peer's finishers wait for that
+// page t + 2 before they take their page t + 3 out of staging, which the
+// peer's sender needs before it ships page t + 4 into the buffer page t used.
 static_assert(XBUF >= 4, "the exchange needs four buffers (see above)");
 constexpr int SG_BYTES = MAX_OWN * CHUNK_BYTES;
 constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
@@ -84,11 +85,15 @@ constexpr int OFF_X = 0;
 constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
 constexpr int OFF_SG = OFF_XS + X_BYTES;
 constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
-constexpr int OFF_BAR = OFF_VG + VGROUPS * VG_BYTES;
-constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 9;
+constexpr int OFF_MH = OFF_VG + VGROUPS * VG_BYTES;  // half-row maxima [2][2][128] fp32 (sums reuse a slot)
+constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
+constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 9 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + slack to align the base to 1024
+// No slack for aligning the base: the kernel has no static shared memory, so
+// its dynamic block starts on a 1024-byte boundary (the kernel checks this
+// and reports MLA_ERR_UNSUPPORTED otherwise).
+constexpr size_t SMEM_BYTES = SMEM_USED;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA can have");
 
 struct Params {
@@ -161,8 +166,11 @@ __device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
+    if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
   uint64_t* sg_full = x_full + XBUF;     // [SGROUPS]
@@ -177,7 +185,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* o_free = s_full + 5;
   uint64_t* final_bar = s_full + 6;
   uint64_t* xs_full = s_full + 7;  // the sender has staged a page's partial
-  uint64_t* xs_free = s_full + 8;  // the finisher has taken it out of the staging block
+  uint64_t* xs_free = s_full + 8;  // the finishers have taken it out of the staging block
+  uint64_t* pair_bars = s_full + 9;  // [4]: the two finisher warps of a lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -203,13 +212,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int i = 0; i < XBUF; ++i) mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);   // sender
-    mbar_init(p_ready, 128);  // finisher
+    mbar_init(p_ready, 256);  // finishers
     mbar_init(pv_done, 1);
     mbar_init(q_ready, 128);  // sender
-    mbar_init(o_free, 128);   // finisher
+    mbar_init(o_free, 256);   // finishers
     mbar_init(final_bar, 2);  // one commit per issuer warp
     mbar_init(xs_full, 128);
-    mbar_init(xs_free, 128);
+    mbar_init(xs_free, 256);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -360,11 +370,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // The two work on consecutive pages at once, so the exchange of page t+1
     // overlaps the softmax of page t, and no row is split between threads.
     const bool sender = warp < 8;
-    const int r = tid - (sender ? 128 : 256);
+    const int h = warp >= 12 ? 1 : 0;  // finisher half: keys [32h, 32h + 32)
+    const int r = tid - (sender ? 128 : 256 + 128 * h);
     const int lane = tid & 31;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O;
-    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P;
+    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P + 16 * h;
     uint8_t* sX = smem + OFF_X;
     uint8_t* sXS = smem + OFF_XS;
     bool ok = true;
@@ -415,16 +426,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (!(ok = wait_all(s_full, tg & 1))) break;
           tc_fence_after();
           uint32_t cur[32];
-          {
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tS, v0);
-            tmem_ld32(tS + 32, v1);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld32(tS + 32 * half, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              cur[j] = pack_bf16x2(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1]));
-              cur[16 + j] = pack_bf16x2(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1]));
-            }
+            for (int j = 0; j < 16; ++j)
+              cur[16 * half + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
           }
           tc_fence_before();
           mbar_arrive(s_free);
@@ -455,6 +464,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
     } else {
+      // Two finisher warpgroups: half h owns keys [32h, 32h + 32) of every
+      // row and half of O's columns; the two threads of a row (their warps
+      // share a lane quarter) agree on the row max through a bounded
+      // 64-arrival mbarrier.
+      uint64_t* pair_bar = &pair_bars[warp & 3];
+      uint32_t pair_phase = 0;
+      auto pair_sync = [&]() -> bool {
+        mbar_arrive(pair_bar);
+        bool r_ok = mbar_wait(pair_bar, pair_phase & 1, abort_flag, a.err);
+        ++pair_phase;
+        return __all_sync(0xffffffffu, r_ok);
+      };
+      float* mh = reinterpret_cast<float*>(smem + OFF_MH);
+      const int hc0 = h * (dh / 64), hc1 = hc0 + dh / 64;  // this half's 32-column chunks of O
       Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
       Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
       uint8_t* sV = smem + OFF_VG;
@@ -469,20 +492,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           // This CTA's partial, staged by the sender; the block goes straight
           // back to it.
           if (!(ok = wait_all(xs_full, tg & 1))) break;
-          uint4 own4[8];
+          uint4 own4[4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) own4[u] = *reinterpret_cast<const uint4*>(sXS + x_off(r, u));
+          for (int u = 0; u < 4; ++u) own4[u] = *reinterpret_cast<const uint4*>(sXS + x_off(r, 4 * h + u));
           mbar_arrive(xs_free);
           // The peer's partial (its bytes complete this CTA's barrier).
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_full[xb], (tg / XBUF) & 1, abort_flag, a.err,
                                                        2000000000ull, true, true))))
             break;
-          float s[64];
+          float s[32];
           {
             const uint8_t* src = sX + xb * X_BYTES;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, u));
+            for (int u = 0; u < 4; ++u) {
+              const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, 4 * h + u));
               const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
               const uint32_t mw[4] = {own4[u].x, own4[u].y, own4[u].z, own4[u].w};
 #pragma unroll
@@ -494,25 +517,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               }
             }
           }
-          const int valid = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
-          if (valid < KT) {
+          const int valid_all = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
+          const int valid = valid_all - 32 * h;             // valid keys among this half's 32
+          if (valid < 32) {
 #pragma unroll
-            for (int j = 0; j < KT; ++j)
+            for (int j = 0; j < 32; ++j)
               if (j >= valid) s[j] = -INFINITY;
           }
           float mt;
           {
-            float mx[32];
+            float mx[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx[j] = fmaxf(s[j], s[j + 32]);
+            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
 #pragma unroll
-            for (int w2 = 16; w2 >= 1; w2 >>= 1)
+            for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
               for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-            mt = mx[0];
+            float* slot = mh + (tg & 1) * 256;
+            slot[h * 128 + r] = mx[0];
+            if (!(ok = pair_sync())) break;
+            mt = fmaxf(slot[r], slot[128 + r]);
           }
           // Running max with lazy rescaling: O and l stay relative to m_used
-          // until a page's max exceeds it by more than 2^8.
+          // until a page's max exceeds it by more than 2^8.  Both halves take
+          // the same decision from the same two numbers.
           bool resc = false;
           float scale = 1.f;
           if (i == 0) {
@@ -523,17 +551,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             m_used = mt;
             resc = true;
           }
-          uint32_t pk[32];
+          uint32_t pk[16];
           float psum;
           {
-            float ps[16];
+            float ps[8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) ps[u] = 0.f;
+            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
-            for (int u = 0; u < 32; ++u)
-              pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u & 15]);
+            for (int u = 0; u < 16; ++u)
+              pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u & 7]);
 #pragma unroll
-            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+            for (int w2 = 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
               for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
             psum = ps[0];
@@ -544,7 +572,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tc_fence_after();
           }
           if (__any_sync(0xffffffffu, resc)) {
-            for (int cc = 0; cc < dh / 32; ++cc) {
+            for (int cc = hc0; cc < hc1; ++cc) {
               uint32_t v[32];
               tmem_ld32(tO + cc * 32, v);
               tmem_ld_wait();
@@ -554,19 +582,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             l *= scale;
           }
-          tmem_st32(tP, pk);
+          tmem_st16(tP, pk);
           tmem_st_wait();
           l += psum;
-          if (valid < KT) {
+          if (valid_all < KT) {
             // Keys past the end: P is 0 there, but 0 * NaN would still poison
             // O, so clear those rows of this page's latent chunks (once they
             // have landed).
             if (!(ok = wait_all(&vg_full[tg % VGROUPS], (tg / VGROUPS) & 1))) break;
             uint8_t* gb = sV + (tg % VGROUPS) * VG_BYTES;
-            const int rows = KT - valid, units = rows * 8 * npv;
-            for (int x = r; x < units; x += 128) {
+            const int rows = KT - valid_all, units = rows * 8 * npv;
+            for (int x = r + 128 * h; x < units; x += 256) {
               const int q = x / (rows * 8), rem = x - q * rows * 8;
-              *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+              *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
@@ -578,11 +606,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           // ---- epilogue of the segment ----
           if (!(ok = wait_all(pv_done, tg & 1))) break;
           tc_fence_after();
+          // Row sum: both halves add the two partial sums in the same order.
+          // The sums borrow the max slot of the previous page: the partner
+          // read that page's maxima before the last pair sync, and the next
+          // page's maxima go there only after the second sync below.
+          float* ls = mh + ((tg + 1) & 1) * 256;
+          ls[h * 128 + r] = l;
+          if (!(ok = pair_sync())) break;
+          const float lrow = ls[r] + ls[128 + r];
+          if (!(ok = pair_sync())) break;
           // A whole row block is normalised into obar (bf16); a piece of a
           // split row block leaves its unnormalised sum and (m, l) in its slot.
           const bool whole = g.slot < 0;
-          const float inv = 1.f / l;
-          for (int cc = 0; cc < dh / 32; ++cc) {
+          const float inv = 1.f / lrow;
+          for (int cc = hc0; cc < hc1; ++cc) {
             uint32_t v[32];
             tmem_ld32(tO + cc * 32, v);
             tmem_ld_wait();
@@ -608,9 +645,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               }
             }
           }
-          if (!whole && rank == 0 && r < a.n_h) {
+          if (!whole && rank == 0 && h == 0 && r < a.n_h) {
             a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 0] = m_used;
-            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = l;
+            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = lrow;
           }
           tc_fence_before();
           mbar_arrive(o_free);

@@ -7,7 +7,7 @@
 namespace mla {
 
 // Bits OR-ed into the workspace error word by device-side checks.
-enum DeviceErr : int { kErrBounds = 1, kErrTimeout = 2 };
+enum DeviceErr : int { kErrBounds = 1, kErrTimeout = 2, kErrLayout = 4 };
 
 __device__ __forceinline__ void flag_error(int* err_word, int bit) {
   if (err_word) atomicOr(err_word, bit);

@@ -685,6 +685,7 @@ mla_status mla_get_error(const void* workspace, cudaStream_t stream) {
   cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (word & kErrLayout) return MLA_ERR_UNSUPPORTED;
   if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
   if (word & kErrBounds) return MLA_ERR_DEVICE_BOUNDS;
   return MLA_OK;

@@ -192,8 +192,9 @@ mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_
  * ------------------------------------------------------------------------- */
 /* Waits for `stream`, then returns the error recorded on the device by the
  * most recent call that used `workspace` (MLA_OK if none): MLA_ERR_TIMEOUT
- * (a bounded wait gave up) or MLA_ERR_DEVICE_BOUNDS (a page id or length out
- * of range). */
+ * (a bounded wait gave up), MLA_ERR_DEVICE_BOUNDS (a page id or length out
+ * of range), or MLA_ERR_UNSUPPORTED (the device placed the attention
+ * kernel's shared memory off the 1024-byte alignment it relies on). */
 mla_status mla_get_error(const void* workspace, cudaStream_t stream);
 
 /* Static, human-readable name of a status code. */
