@@ -17,11 +17,13 @@
 // B200 layout.  TMEM (128 lanes x 512 fp32 columns per SM) cannot hold the
 // 128 x 512 fp32 latent accumulator of one token next to anything else, so
 // the two CTAs of a cluster split the columns of the cache row:
-//   rank 0: latent columns [0, d_c/2)
-//   rank 1: latent columns [d_c/2, d_c) and the RoPE key columns.
-// Each CTA streams only its own columns of every page (no byte is read twice),
-// computes the partial score over them (all of its Q slice is the TMEM A
-// operand), and sends the partial, rounded to bf16, to its peer through
+//   rank 0: latent columns [0, d_c/2) and the first ra RoPE-key columns
+//   rank 1: latent columns [d_c/2, d_c) and the other rb = d_r - ra,
+// with ra = 16 * (d_r / 32) so that both score shares are whole 16-column MMA
+// steps and, for d_r = 32 or 64, equal (the score MMA is the longest tensor
+// job per page).  Each CTA streams only its own columns of every page (no byte
+// is read twice), computes the partial score over them (all of its Q slice is
+// the TMEM A operand), and sends the partial, rounded to bf16, to its peer through
 // distributed shared memory.  Both CTAs add the two bf16 partials in fp32 --
 // the same two numbers, so both see bit-identical scores and run identical
 // softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
@@ -29,8 +31,9 @@
 // P [480, 512).
 //
 // Shared memory (128-byte swizzled 64 x 64 chunks, loaded by TMA):
-//   score ring, 2 slots: this CTA's columns of a page (<= 5 chunks), freed as
-//     soon as the page's score MMA completes;
+//   score ring, 2 slots: this CTA's columns of a page (its latent chunks and
+//     its RoPE share, loaded with a 16- or 32-column box swizzled to 32 or 64
+//     bytes), freed as soon as the page's score MMA completes;
 //   latent ring, 2 slots: the page's latent columns again (4 chunks) for
 //     P*V, freed by P*V.  The second read is an L2 hit (the first was a few
 //     microseconds earlier), so HBM still sees every byte once; decoupling
@@ -62,8 +65,8 @@ using namespace sm100;
 constexpr int THREADS = 512;
 constexpr int KT = 64;                        // keys per tile (one page)
 constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
-constexpr int MAX_OWN = 5;                    // score chunks per CTA per page
 constexpr int MAX_PV = 4;                     // latent chunks per CTA per page (d_c <= 512)
+constexpr int MAX_ROPE = 32;                  // RoPE-key columns per CTA (d_r <= 64)
 constexpr int SGROUPS = 2;                    // score ring: a page's own columns, freed by its score MMA
 constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
 constexpr int XBUF = 4;                       // exchange buffers per CTA
@@ -74,7 +77,8 @@ constexpr int XBUF = 4;                       // exchange buffers per CTA
 // page t + 2 before they take their page t + 3 out of staging, which the
 // peer's sender needs before it ships page t + 4 into the buffer page t used.
 static_assert(XBUF >= 4, "the exchange needs four buffers (see above)");
-constexpr int SG_BYTES = MAX_OWN * CHUNK_BYTES;
+constexpr int ROPE_OFF = MAX_PV * CHUNK_BYTES;  // a score slot: latent chunks, then the RoPE share
+constexpr int SG_BYTES = ROPE_OFF + KT * MAX_ROPE * 2;
 constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
@@ -98,8 +102,8 @@ static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA can 
 
 struct Params {
   AttnArgs a;
-  int nkc;  // 64-column chunks per cache row (ceil(d_cr / 64))
-  int npv;  // latent chunks per CTA (d_c / 128)
+  int npv;     // latent chunks per CTA (d_c / 128)
+  int ra, rb;  // RoPE-key columns scored by rank 0 and rank 1 (multiples of 16, ra + rb = d_r)
 };
 
 // 2^x with the MUFU ex2 instruction (flush-to-zero; ~2 ulp), used for the
@@ -165,7 +169,8 @@ constexpr int X_WARP_BYTES = 32 * KT * 2;
 __device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap rmap16,
+                   const __grid_constant__ CUtensorMap rmap32, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
     if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
@@ -194,9 +199,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
   const int w = blockIdx.x >> 1;
   const AttnArgs& a = p.a;
-  const int nkc = p.nkc, npv = p.npv, dh = npv * 64;
-  const int c_lo = rank ? npv : 0;                 // first chunk this CTA loads
-  const int n_own = rank ? nkc - npv : npv;        // chunks this CTA loads per page
+  const int npv = p.npv, dh = npv * 64;
+  const int c_lo = (int)rank * npv;                // first latent chunk of this CTA
+  const int rw = rank ? p.rb : p.ra;               // RoPE-key columns this CTA scores (0, 16 or 32)
+  const int rx = a.d_c + (rank ? p.ra : 0);        // and the first of them
+  const CUtensorMap* rmap = rw == 32 ? &rmap32 : &rmap16;
   const Seg* segs = a.sched.segs;
   const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
@@ -228,7 +235,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
-  if (tid == 0) tma_prefetch_desc(&tmap);
+  if (tid == 0) {
+    tma_prefetch_desc(&tmap);
+    if (rw) tma_prefetch_desc(rmap);
+  }
   __syncthreads();
   cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
@@ -243,8 +253,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // streams, the next page id while this page waits for its ring slot.
     const bool score_ring = warp == 0;
     const int nring = score_ring ? SGROUPS : VGROUPS;
-    const int nchunk = score_ring ? n_own : npv;
     const int ring_bytes = score_ring ? SG_BYTES : VG_BYTES;
+    const int rope_cols = score_ring ? rw : 0;
     uint8_t* ring = smem + (score_ring ? OFF_SG : OFF_VG);
     uint64_t* full = score_ring ? sg_full : vg_full;
     uint64_t* empty = score_ring ? sg_empty : vg_empty;
@@ -275,9 +285,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(&full[gs], nchunk * CHUNK_BYTES);
-          for (int q = 0; q < nchunk; ++q)
+          mbar_arrive_expect_tx(&full[gs], npv * CHUNK_BYTES + rope_cols * KT * 2);
+          for (int q = 0; q < npv; ++q)
             tma_load_2d(ring + gs * ring_bytes + q * CHUNK_BYTES, &tmap, (c_lo + q) * 64, page * KT, &full[gs]);
+          if (rope_cols) tma_load_2d(ring + gs * ring_bytes + ROPE_OFF, rmap, rx, page * KT, &full[gs]);
         }
         __syncwarp();
         ++cnt;
@@ -315,12 +326,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
           if (elect_one()) {
             const uint32_t gb = sSG + gs * SG_BYTES;
-            for (int q = 0; q < n_own; ++q) {
+            for (int q = 0; q < npv; ++q) {
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 mma_ts(tS, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
                        (q | k) ? 1u : 0u);
             }
+            // The RoPE share: rows of rw * 2 bytes, swizzled to that width.
+            for (int k = 0; k < rw / 16; ++k)
+              mma_ts(tS, tQ + npv * 32 + k * 8,
+                     sdesc_swz(gb + ROPE_OFF + k * 32, 8 * rw * 2, rw == 32 ? kSwizzle64 : kSwizzle32), idS, 1u);
             tc_commit(s_full);
             tc_commit(&sg_empty[gs]);  // the score ring slot is free once its MMAs are done
           }
@@ -392,18 +407,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       auto load_q = [&](int rb) {
         const uint4* src =
             (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
-        for (int q = 0; q < n_own; ++q) {
+        for (int q = 0; q < npv; ++q) {
           uint32_t wv[32];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int col = (c_lo + q) * 64 + u * 8;
-            uint4 v = (src && col < a.d_cr) ? __ldg(src + col / 8) : make_uint4(0, 0, 0, 0);
+            uint4 v = src ? __ldg(src + ((c_lo + q) * 64 + u * 8) / 8) : make_uint4(0, 0, 0, 0);
             wv[4 * u + 0] = v.x;
             wv[4 * u + 1] = v.y;
             wv[4 * u + 2] = v.z;
             wv[4 * u + 3] = v.w;
           }
           tmem_st32(tQ + q * 32, wv);
+        }
+        if (rw) {
+          uint32_t wv[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 v = (src && u * 8 < rw) ? __ldg(src + (rx + u * 8) / 8) : make_uint4(0, 0, 0, 0);
+            wv[4 * u + 0] = v.x;
+            wv[4 * u + 1] = v.y;
+            wv[4 * u + 2] = v.z;
+            wv[4 * u + 3] = v.w;
+          }
+          if (rw == 32) {
+            tmem_st16(tQ + npv * 32, wv);
+          } else {
+            uint32_t w8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w8[j] = wv[j];
+            tmem_st8(tQ + npv * 32, w8);
+          }
         }
         tmem_st_wait();
         tc_fence_before();

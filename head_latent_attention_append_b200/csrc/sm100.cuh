@@ -194,6 +194,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (2ull << 61) /* 128-byte swizzle */;
 }
 
+// Same for a K-major tile whose rows are 64 or 32 bytes, swizzled to that
+// width (layout type 4 = 64-byte, 6 = 32-byte swizzle); `sbo` is the stride of
+// 8-row groups (8 x the row bytes).
+constexpr uint64_t kSwizzle64 = 4, kSwizzle32 = 6;
+__device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t sbo, uint64_t layout) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) /* leading offset: unused when swizzled */ |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (layout << 61);
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4)                                   /* D: f32 */
