@@ -18,8 +18,8 @@ using namespace sm100;
 
 constexpr int BM = 128;      // weight rows per tile
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row)
-constexpr int STAGES = 4;
-constexpr int THREADS = 128;
+constexpr int EPI_WARPS = 16;  // four per TMEM lane quarter, each draining a quarter of the tile's columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0: TMA producer; warp 1: TMEM + MMA issue; then the epilogue
 
 struct Args {
   int Mw;                    // weight rows per batch entry (output columns)
@@ -29,46 +29,71 @@ struct Args {
   int a_batch_rows;          // row offset of batch entry b in A = b * a_batch_rows
   int b_is_3d;               // B map has a per-batch (head) dimension
   float* partial;            // [batch][tiles_m][tiles_n][splits][BN][BM] when splits > 1
+  int tiles_m, tiles_n, batch;
 };
 
 template <int BN>
+__host__ __device__ constexpr int stages() {
+  return BN == 64 ? 8 : 6;
+}
+template <int BN>
 constexpr size_t smem_bytes() {
-  return (size_t)STAGES * (BM + BN) * BK * 2 + 1024 + 256;
+  return (size_t)stages<BN>() * (BM + BN) * BK * 2 + 1024 + 256;
 }
 
+// Persistent and warp-specialised: each CTA walks work items (weight tile,
+// token tile, batch entry, K split) item = blockIdx.x, += gridDim.x.  The
+// producer streams every item's K steps through an stages<BN>()-deep ring
+// without stopping between items; the MMA warp accumulates item i into one
+// of two TMEM accumulators while the epilogue warps drain the other, so a
+// tile's epilogue overlaps the next tile's loads and MMAs.
 template <int BN, class Epi>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const Args g, const Epi epi) {
+  constexpr int STAGES = stages<BN>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE = A_BYTES + B_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
   uint64_t* empty = full + STAGES;
-  uint64_t* done = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* drained = acc_empty + 2;     // every MMA this CTA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int tiles_n = gridDim.y;
-  const int bz = blockIdx.z / g.splits, split = blockIdx.z % g.splits;
-  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
-  const int k_begin = split * g.kchunk;
-  const int k_end = min(g.K, k_begin + g.kchunk);
-  const int nk = k_end > k_begin ? (k_end - k_begin + BK - 1) / BK : 0;
+  const int per_z = g.tiles_m * g.tiles_n;
+  const int items = per_z * g.batch * g.splits;
+  auto decode = [&](int item, int& bz, int& split, int& tm, int& tn) {
+    const int z = item / per_z, rem = item - z * per_z;
+    bz = z / g.splits;
+    split = z - bz * g.splits;
+    tm = rem % g.tiles_m;
+    tn = rem / g.tiles_m;
+  };
+  auto ksteps = [&](int split) {
+    const int k_begin = split * g.kchunk, k_end = min(g.K, k_begin + g.kchunk);
+    return k_end > k_begin ? (k_end - k_begin + BK - 1) / BK : 0;
+  };
 
   if (tid == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 32 * EPI_WARPS);
+    }
+    mbar_init(drained, 1);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN < 32 ? 32 : BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   __syncthreads();
@@ -76,84 +101,121 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 0) {
-    // TMA producer.
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % STAGES;
-      if (!mbar_wait_warp(&empty[s], ((kt / STAGES) & 1) ^ 1, abort_flag, nullptr)) break;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&full[s], STAGE);
-        const int k = k_begin + kt * BK;
-        tma_load_2d(smem + s * STAGE, &mapA, k, bz * g.a_batch_rows + m0, &full[s]);
-        if (g.b_is_3d) tma_load_3d(smem + s * STAGE + A_BYTES, &mapB, k, bz, n0, &full[s]);
-        else tma_load_2d(smem + s * STAGE + A_BYTES, &mapB, k, n0, &full[s]);
+    // TMA producer: runs ahead across items as far as the ring allows.
+    uint32_t cnt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      int bz, split, tm, tn;
+      decode(item, bz, split, tm, tn);
+      const int nk = ksteps(split);
+      for (int kt = 0; kt < nk; ++kt, ++cnt) {
+        const int s = cnt % STAGES;
+        if (!(ok = mbar_wait_warp(&empty[s], ((cnt / STAGES) & 1) ^ 1, abort_flag, nullptr))) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full[s], STAGE);
+          const int k = split * g.kchunk + kt * BK;
+          tma_load_2d(smem + s * STAGE, &mapA, k, bz * g.a_batch_rows + tm * BM, &full[s]);
+          if (g.b_is_3d) tma_load_3d(smem + s * STAGE + A_BYTES, &mapB, k, bz, tn * BN, &full[s]);
+          else tma_load_2d(smem + s * STAGE + A_BYTES, &mapB, k, tn * BN, &full[s]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
+    }
+    if (*abort_flag) {
+      // Let every copy already issued land before the CTA can exit.
+      for (uint32_t q = 0; q < (uint32_t)STAGES && q < cnt; ++q) {
+        const uint32_t last = q + STAGES * ((cnt - 1 - q) / STAGES);
+        mbar_wait_warp(&full[q], (last / STAGES) & 1, abort_flag, nullptr, 50000000ull, false);
+      }
     }
   } else if (warp == 1) {
     // MMA issuer.
     const uint32_t idesc = idesc_bf16(BM, BN, 0, 0);
     const uint32_t s0 = smem_u32(smem);
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % STAGES;
-      if (!mbar_wait_warp(&full[s], (kt / STAGES) & 1, abort_flag, nullptr)) break;
+    uint32_t cnt = 0, li = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++li) {
+      int bz, split, tm, tn;
+      decode(item, bz, split, tm, tn);
+      const int nk = ksteps(split);
+      const uint32_t acc = li & 1;
+      if (!(ok = mbar_wait_warp(&acc_empty[acc], ((li >> 1) & 1) ^ 1, abort_flag, nullptr))) break;
       tc_fence_after();
-      if (elect_one()) {
-        const uint32_t a = s0 + s * STAGE, b = a + A_BYTES;
+      for (int kt = 0; kt < nk; ++kt, ++cnt) {
+        const int s = cnt % STAGES;
+        if (!(ok = mbar_wait_warp(&full[s], (cnt / STAGES) & 1, abort_flag, nullptr))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t a = s0 + s * STAGE, b = a + A_BYTES;
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          mma_ss(tbase, sdesc_sw128(a + k * 32, 16, 1024), sdesc_sw128(b + k * 32, 16, 1024), idesc,
-                 (kt | k) ? 1u : 0u);
-        tc_commit(&empty[s]);
+          for (int k = 0; k < BK / 16; ++k)
+            mma_ss(tbase + acc * BN, sdesc_sw128(a + k * 32, 16, 1024), sdesc_sw128(b + k * 32, 16, 1024), idesc,
+                   (kt | k) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        __syncwarp();
       }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&acc_full[acc]);
       __syncwarp();
     }
-    if (elect_one()) tc_commit(done);
+    // TMEM is freed only after the last MMA, even on an abandoned run.
+    if (elect_one()) tc_commit(drained);
     __syncwarp();
-  }
-
-  // Epilogue (all four warps): thread r holds weight row m0 + r for the BN
-  // tokens of the tile.
-  mbar_wait(done, 0, abort_flag, nullptr, 2000000000ull, false);
-  __syncwarp();
-  tc_fence_after();
-  const int r = tid;
-  const uint32_t taddr = tbase + ((uint32_t)(warp * 32) << 16);
-  const int col = m0 + r;
-  const int ntiles = gridDim.x * tiles_n;
-  float* part = nullptr;
-  if (g.splits > 1)
-    part = g.partial + (((long long)bz * ntiles + blockIdx.x * tiles_n + blockIdx.y) * g.splits + split) *
-                           (long long)(BN * BM);
-  // Eight token columns at a time (a short body keeps the functor's code
-  // small enough for the instruction cache).
+    mbar_wait_warp(drained, 0, abort_flag, nullptr, 50000000ull, false);
+  } else {
+    // Epilogue (warps 2 .. 2 + EPI_WARPS - 1): thread r holds weight row
+    // tm * BM + r of the item; a warp reaches the TMEM lanes of its quarter
+    // and drains one quarter of the item's BN token columns.
+    const int q = warp & 3, r = q * 32 + (tid & 31);
+    const int part = (warp - 2) / 4, c_lo = part * (BN / 4), c_hi = c_lo + BN / 4;
+    uint32_t li = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++li) {
+      int bz, split, tm, tn;
+      decode(item, bz, split, tm, tn);
+      const int nk = ksteps(split);
+      const uint32_t acc = li & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (li >> 1) & 1, abort_flag, nullptr))) break;
+      tc_fence_after();
+      const uint32_t taddr = tbase + acc * BN + ((uint32_t)(q * 32) << 16);
+      const int col = tm * BM + r;
+      float* pdst = nullptr;
+      if (g.splits > 1)
+        pdst = g.partial + (((long long)bz * per_z + tm * g.tiles_n + tn) * g.splits + split) * (long long)(BN * BM);
+      // Eight token columns at a time (a short body keeps the functor's code
+      // small enough for the instruction cache).
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 8) {
-    uint32_t v[8];
-    if (nk > 0) {
-      tmem_ld8(taddr + c0, v);
-      tmem_ld_wait();
-    } else {
+      for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
+        uint32_t v[8];
+        if (nk > 0) {
+          tmem_ld8(taddr + c0, v);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0u;
-    }
-    if (part) {
+          for (int j = 0; j < 8; ++j) v[j] = 0u;
+        }
+        if (pdst) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) __stcg(part + (c0 + j) * BM + r, __uint_as_float(v[j]));
-    } else {
+          for (int j = 0; j < 8; ++j) __stcg(pdst + (c0 + j) * BM + r, __uint_as_float(v[j]));
+        } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float mine = __uint_as_float(v[j]);
-        const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-        const int tok = n0 + c0 + j;
-        if ((r & 1) == 0 && col < g.Mw && tok < g.Nt) epi(bz, tok, col, mine, other);
+          for (int j = 0; j < 8; ++j) {
+            const float mine = __uint_as_float(v[j]);
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const int tok = tn * BN + c0 + j;
+            if ((r & 1) == 0 && col < g.Mw && tok < g.Nt) epi(bz, tok, col, mine, other);
+          }
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, BN < 32 ? 32 : BN);
+    tmem_dealloc(tbase, 2 * BN);
   }
 }
 
@@ -161,7 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 // epilogue.  Grid: (tiles_m, tiles_n * BN / 8, batch); block 256 = 8 tokens x
 // 32 lanes; each thread owns two column pairs of one token and keeps all of
 // their split loads in flight.
-constexpr int MAX_SPLITS = 8;
+constexpr int MAX_SPLITS = 32;
 template <int BN, class Epi>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const Args g, const Epi epi) {
   const int bz = blockIdx.z, slices = BN / 8;

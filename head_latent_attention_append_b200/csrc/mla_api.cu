@@ -265,19 +265,23 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   }
   const int tm = ceil_div(N, gemm_tc::BM), tn = ceil_div(M, BN), tiles = tm * tn * batch;
   const int nk = ceil_div(K, gemm_tc::BK);
+  // Few output tiles (decode): split K so that about two work items per SM
+  // keep every SM streaming weights; the reduce kernel sums the splits in
+  // order and runs the epilogue.
   int splits = 1;
   const int sms = num_sms();
-  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), ceil_div(sms, tiles));
+  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), ceil_div(2 * sms, tiles));
   while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
   const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
   splits = ceil_div(K, kchunk);
-  gemm_tc::Args g{N, M, K, splits, kchunk, N, x3d ? 1 : 0, partial};
+  gemm_tc::Args g{N, M, K, splits, kchunk, N, x3d ? 1 : 0, partial, tm, tn, batch};
   const size_t smem = gemm_tc::smem_bytes<BN>();
   auto kfn = gemm_tc::gemm_tc_kernel<BN, Epi>;
   cudaError_t e = set_smem_once(kfn, smem);
   if (e != cudaSuccess) return e;
   ++g_launches;
-  kfn<<<dim3(tm, tn, batch * splits), gemm_tc::THREADS, smem, st>>>(mapW, mapX, g, epi);
+  const int items = tiles * splits;
+  kfn<<<dim3(std::min(items, sms)), gemm_tc::THREADS, smem, st>>>(mapW, mapX, g, epi);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (splits > 1) {
     ++g_launches;
