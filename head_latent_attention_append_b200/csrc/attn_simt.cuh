@@ -170,9 +170,19 @@ inline size_t smem_bytes(int HG, int d_cr) {
 // ------------------------------------------------------------ combine -----
 // Merges the partial slots of each split row block (log-sum-exp in base 2):
 //   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  obar = sum_s 2^(m_s - m) O_s / l.
-// Block = (split row block, 8 heads), one warp per head, lanes across the
-// latent columns.  Slots are visited in segment order, so the result is
-// deterministic.
+// Block = (split row block, 8 heads), one warp per head.  Lane k gathers the
+// (slot, m, l) of segments k, k + 32, ...; the warp reduces them with
+// shuffles, then each lane accumulates four consecutive latent columns of
+// each 128-column chunk (d_c <= 512) with 16-byte loads.  Slots are added in
+// segment order, so the result is deterministic.
+__device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
   const Sched& S = a.sched;
@@ -182,32 +192,57 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (h >= a.n_h) return;
   const int s0 = S.rb_seg_first[rb], s1 = S.rb_seg_first[rb + 1];
+  // Row max and sum over the segments.
   float m = -INFINITY;
-  for (int s = s0; s < s1; ++s) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
+  for (int s = s0 + lane; s < s1; s += 32) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float l = 0.f;
-  for (int s = s0; s < s1; ++s) {
+  for (int s = s0 + lane; s < s1; s += 32) {
     const float* ml = a.part_ml + ((long long)S.segs[s].slot * a.n_h + h) * 2;
     l += exp2f(ml[0] - m) * ml[1];
   }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   const float inv = 1.f / l;
   T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
-  for (int j0 = 0; j0 < a.d_c; j0 += 128) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = s0; s < s1; ++s) {
-      const int slot = S.segs[s].slot;
-      const float wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
-      const float* src = a.part_o + ((long long)slot * a.n_h + h) * a.d_c + j0;
+  // All four 128-column chunks (d_c <= 512) at once, so a warp's loads are in
+  // flight together.
+  float4 acc[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = q * 32 + lane;
-        if (j0 + j < a.d_c) acc[q] += wgt * __ldcg(src + j);
+  for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sb = s0; sb < s1; sb += 32) {
+    // Lane k holds segment sb + k's slot and weight; broadcast in order.
+    int slot = 0;
+    float wgt = 0.f;
+    if (sb + lane < s1) {
+      slot = S.segs[sb + lane].slot;
+      wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
+    }
+    const int cnt = min(32, s1 - sb);
+    for (int k = 0; k < cnt; ++k) {
+      const int sl = __shfl_sync(0xffffffffu, slot, k);
+      const float w = __shfl_sync(0xffffffffu, wgt, k);
+      const float* src = a.part_o + ((long long)sl * a.n_h + h) * a.d_c;
+      float4 v[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = c * 128 + 4 * lane;
+        v[c] = j < a.d_c ? __ldcg(reinterpret_cast<const float4*>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[c].x += w * v[c].x;
+        acc[c].y += w * v[c].y;
+        acc[c].z += w * v[c].z;
+        acc[c].w += w * v[c].w;
       }
     }
+  }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = j0 + q * 32 + lane;
-      if (j < a.d_c) out[j] = from_f32<T>(acc[q] * inv);
-    }
+  for (int c = 0; c < 4; ++c) {
+    const int j = c * 128 + 4 * lane;
+    if (j < a.d_c) store4(out + j, acc[c].x * inv, acc[c].y * inv, acc[c].z * inv, acc[c].w * inv);
   }
 }
 

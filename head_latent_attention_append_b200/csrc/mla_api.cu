@@ -438,7 +438,9 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   {
     SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
     ++g_launches;
-    sched_kernel<<<1, 1024, 0, st>>>(sa);
+    const size_t sched_smem = R + 1 <= kSchedSmemRb ? sizeof(int) * (size_t)(R + 1) : 0;
+    if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
+    sched_kernel<<<1, 1024, sched_smem, st>>>(sa);
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (5) attention on the latent cache, (6) combine of split row blocks.

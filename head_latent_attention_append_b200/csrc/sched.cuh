@@ -114,10 +114,17 @@ __device__ __forceinline__ int find_le(const int* a, int n, int x) {
   return lo;
 }
 
+// Row blocks whose tile offsets the schedule keeps in shared memory (the
+// binary searches below then cost no global round trips); beyond this they
+// stay in global memory.
+constexpr int kSchedSmemRb = 16384;
+
 __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
+  extern __shared__ int sched_smem[];
   const int tid = threadIdx.x, T = blockDim.x;
   const int R = a.R, W = a.W;
-  int* ts = a.s.tile_start;
+  const bool in_smem = R + 1 <= kSchedSmemRb;
+  int* ts = in_smem ? sched_smem : a.s.tile_start;
   for (int rb = tid; rb < R; rb += T)
     ts[rb] = ceil_div(rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, a.err), a.tile);
   __syncthreads();
@@ -159,6 +166,8 @@ __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
     }
   }
   if (tid == 0) a.s.rb_seg_first[R] = nseg;
+  if (in_smem)
+    for (int i = tid; i <= R; i += T) a.s.tile_start[i] = ts[i];
   __syncthreads();
 
   // Row blocks with more than one segment.  Such a row block starts with a
