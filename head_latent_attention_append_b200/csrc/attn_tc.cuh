@@ -529,10 +529,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) own4[u] = *reinterpret_cast<const uint4*>(sXS + x_off(r, 4 * h + u));
           mbar_arrive(xs_free);
-          // The peer's partial (its bytes complete this CTA's barrier).
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_full[xb], (tg / XBUF) & 1, abort_flag, a.err,
-                                                       2000000000ull, true, true))))
-            break;
+          // The peer's partial: its bulk copy completes this CTA's barrier,
+          // and the phase completing makes the copied bytes visible here.
+          if (!(ok = wait_all(&x_full[xb], (tg / XBUF) & 1))) break;
           float s[32];
           {
             const uint8_t* src = sX + xb * X_BYTES;

@@ -66,34 +66,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Same, acquiring at cluster scope: for phases completed by another CTA of
-// the cluster (remote asynchronous stores).
-__device__ __forceinline__ bool mbar_try_wait_sleep_cluster(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase with the given parity to complete.  Every wait is
 // bounded: after `limit_ns` (or once another thread of the CTA has given up,
 // signalled through *abort) it records kErrTimeout in the error word, raises
 // *abort and returns false, so no thread can spin forever.
 // With honor_abort = false the wait ignores *abort (used to drain work that is
 // already in flight before the CTA exits).
-// With cluster_scope = true the wait acquires at cluster scope.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
-                                          uint64_t limit_ns = 2000000000ull, bool honor_abort = true,
-                                          bool cluster_scope = false) {
-  if (!cluster_scope && mbar_try_wait(bar, parity)) return true;
+                                          uint64_t limit_ns = 2000000000ull, bool honor_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (cluster_scope ? mbar_try_wait_sleep_cluster(bar, parity, 100000u) : mbar_try_wait_sleep(bar, parity, 100000u))
-      return true;
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (honor_abort && *abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
