@@ -66,11 +66,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int per_z = g.tiles_m * g.tiles_n;
   const int items = per_z * g.batch * g.splits;
+  // Weight tiles are walked from the last: when items outnumber CTAs, the
+  // first round takes the high rows, which is where a projection keeps the
+  // columns with the costlier epilogue (the rotated q_R of the query
+  // projection), so that epilogue overlaps the CTA's next main loop.
   auto decode = [&](int item, int& bz, int& split, int& tm, int& tn) {
     const int z = item / per_z, rem = item - z * per_z;
     bz = z / g.splits;
     split = z - bz * g.splits;
-    tm = rem % g.tiles_m;
+    tm = g.tiles_m - 1 - rem % g.tiles_m;
     tn = rem / g.tiles_m;
   };
   auto ksteps = [&](int split) {
@@ -220,38 +224,34 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Sums the split-K partials of every tile in split order and runs the
-// epilogue.  Grid: (tiles_m, tiles_n * BN / 8, batch); block 256 = 8 tokens x
-// 32 lanes; each thread owns two column pairs of one token and keeps all of
-// their split loads in flight.
+// epilogue.  Grid: (2 * tiles_m, tiles_n * BN / 8, batch); block 256 = 8
+// tokens x 32 lanes covering 64 weight rows, each lane one column pair of one
+// token, with all of its split loads in flight.
 constexpr int MAX_SPLITS = 32;
 template <int BN, class Epi>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const Args g, const Epi epi) {
   const int bz = blockIdx.z, slices = BN / 8;
+  const int tile_m = blockIdx.x >> 1, half = blockIdx.x & 1;
   const int tile_n = blockIdx.y / slices, slice = blockIdx.y % slices;
-  const int tiles_n = gridDim.y / slices, ntiles = gridDim.x * tiles_n;
-  const int m0 = blockIdx.x * BM, n0 = tile_n * BN;
-  const float* base =
-      g.partial + ((long long)bz * ntiles + blockIdx.x * tiles_n + tile_n) * g.splits * (long long)(BN * BM);
+  const int m0 = tile_m * BM, n0 = tile_n * BN;
+  const float* base = g.partial + ((long long)bz * g.tiles_m * g.tiles_n + tile_m * g.tiles_n + tile_n) * g.splits *
+                                      (long long)(BN * BM);
   const int tok_l = slice * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
+  const int cp = (half * 32 + (threadIdx.x % 32)) * 2;
+  float2 v[MAX_SPLITS];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int cp = (half * 32 + lane) * 2;
-    float2 v[MAX_SPLITS];
+  for (int s = 0; s < MAX_SPLITS; ++s)
+    if (s < g.splits)
+      v[s] = __ldcg(reinterpret_cast<const float2*>(base + (long long)s * (BN * BM) + tok_l * BM + cp));
+  float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int s = 0; s < MAX_SPLITS; ++s)
-      if (s < g.splits)
-        v[s] = __ldcg(reinterpret_cast<const float2*>(base + (long long)s * (BN * BM) + tok_l * BM + cp));
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-    for (int s = 0; s < MAX_SPLITS; ++s)
-      if (s < g.splits) {
-        s0 += v[s].x;
-        s1 += v[s].y;
-      }
-    const int tok = n0 + tok_l, col = m0 + cp;
-    if (tok < g.Nt && col < g.Mw) epi(bz, tok, col, s0, s1);
-  }
+  for (int s = 0; s < MAX_SPLITS; ++s)
+    if (s < g.splits) {
+      s0 += v[s].x;
+      s1 += v[s].y;
+    }
+  const int tok = n0 + tok_l, col = m0 + cp;
+  if (tok < g.Nt && col < g.Mw) epi(bz, tok, col, s0, s1);
 }
 
 }  // namespace gemm_tc

@@ -285,7 +285,7 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (splits > 1) {
     ++g_launches;
-    gemm_tc::splitk_reduce_kernel<BN, Epi><<<dim3(tm, tn * (BN / 8), batch), 256, 0, st>>>(g, epi);
+    gemm_tc::splitk_reduce_kernel<BN, Epi><<<dim3(2 * tm, tn * (BN / 8), batch), 256, 0, st>>>(g, epi);
     e = cudaGetLastError();
   }
   return e;
