@@ -30,6 +30,32 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
+// Stores eight consecutive elements: one or two 16-byte stores when the
+// address allows, else pairs.
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store_pair(p + 2 * i, v[2 * i], v[2 * i + 1]);
+  }
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+  if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store_pair(p + 2 * i, v[2 * i], v[2 * i + 1]);
+  }
+}
+
 // RoPE on one interleaved pair (x0, x1) = components (2i, 2i+1), rotated by
 // angle pos * theta_i.  The angle is formed and reduced to [-pi, pi] in fp64
 // (positions reach 2^15, where an fp32 angle would be off by ~4e-3 rad); the

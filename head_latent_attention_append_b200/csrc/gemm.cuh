@@ -37,6 +37,13 @@ struct EpiStore {
   __device__ void operator()(int b, int m, int n, float v0, float v1) const {
     store_pair(C + b * strideC + (long long)m * ldc + n, alpha * v0, alpha * v1);
   }
+  // Columns n0 .. n0 + 7 (n0 a multiple of 8) of row m.
+  __device__ void store8(int b, int m, int n0, const float (&v)[8]) const {
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = alpha * v[i];
+    mla::store8(C + b * strideC + (long long)m * ldc + n0, w);
+  }
 };
 
 // Append: columns [0, d_c) are the latent, [d_c, d_c + d_r) the position key,
@@ -74,6 +81,35 @@ struct EpiAppend {
     if (n >= d_c) rope_rotate_pair(v0, v1, p, theta[(n - d_c) >> 1]);
     store_pair(cache + ((long long)page * page_size + p % page_size) * d_cr + n, v0, v1);
   }
+  // Columns n0 .. n0 + 7 of token m (n0 a multiple of 8; d_c is one too, so
+  // the eight are all latent or all position key).
+  __device__ void store8(int, int m, int n0, const float (&v)[8]) const {
+    int s, p;
+    if (seq_idx) {
+      s = seq_idx[m];
+      p = pos[m];
+    } else {
+      s = m / prefill_S;
+      p = m - s * prefill_S;
+    }
+    if (s < 0 || s >= n_seq || p < 0 || p >= max_pages * page_size) {
+      flag_error(err, kErrBounds);
+      return;
+    }
+    int page = page_table[(long long)s * max_pages + p / page_size];
+    if (page < 0 || page >= num_pages) {
+      flag_error(err, kErrBounds);
+      return;
+    }
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = v[i];
+    if (n0 >= d_c) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rope_rotate_pair(w[2 * i], w[2 * i + 1], p, theta[((n0 - d_c) >> 1) + i]);
+    }
+    mla::store8(cache + ((long long)page * page_size + p % page_size) * d_cr + n0, w);
+  }
 };
 
 // Query projection: columns [0, n_h*d_h) are q_C (stored unscaled for the
@@ -100,6 +136,28 @@ struct EpiQProj {
     else p = (kv_len ? kv_len[m / n_q] : uniform_kv_len) - n_q + m % n_q;
     rope_rotate_pair(v0, v1, p, theta[jj >> 1]);
     store_pair(qabs + ((long long)m * qabs_rows + h) * d_cr + d_c + jj, qr_scale * v0, qr_scale * v1);
+  }
+  // Columns n0 .. n0 + 7 of token m (n0 a multiple of 8; n_h*d_h and d_r are
+  // too, so the eight are all q_C or all one head's q_R).
+  __device__ void store8(int, int m, int n0, const float (&v)[8]) const {
+    const int nc = n_h * d_h;
+    if (n0 < nc) {
+      mla::store8(qc + (long long)m * nc + n0, v);
+      return;
+    }
+    const int j = n0 - nc, h = j / d_r, jj = j - h * d_r;
+    int p;
+    if (prefill_S > 0) p = m % prefill_S;
+    else p = (kv_len ? kv_len[m / n_q] : uniform_kv_len) - n_q + m % n_q;
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float x0 = v[2 * i], x1 = v[2 * i + 1];
+      rope_rotate_pair(x0, x1, p, theta[(jj >> 1) + i]);
+      w[2 * i] = qr_scale * x0;
+      w[2 * i + 1] = qr_scale * x1;
+    }
+    mla::store8(qabs + ((long long)m * qabs_rows + h) * d_cr + d_c + jj, w);
   }
 };
 

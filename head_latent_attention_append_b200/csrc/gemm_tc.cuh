@@ -36,9 +36,13 @@ template <int BN>
 __host__ __device__ constexpr int stages() {
   return BN == 64 ? 8 : 6;
 }
+// Per epilogue warp: 8 tokens x 32 rows of fp32, each token's row padded to
+// 36 floats so that the transposed reads fall in different bank groups.
+constexpr int EPI_PITCH = 36;
+constexpr int EPI_STAGE_BYTES = EPI_WARPS * 8 * EPI_PITCH * 4;
 template <int BN>
 constexpr size_t smem_bytes() {
-  return (size_t)stages<BN>() * (BM + BN) * BK * 2 + 1024 + 256;
+  return (size_t)stages<BN>() * (BM + BN) * BK * 2 + EPI_STAGE_BYTES + 1024 + 256;
 }
 
 // Persistent and warp-specialised: each CTA walks work items (weight tile,
@@ -55,7 +59,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE = A_BYTES + B_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
+  float* epi_stage = reinterpret_cast<float*>(smem + STAGES * STAGE);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE + EPI_STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
@@ -170,9 +175,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // Epilogue (warps 2 .. 2 + EPI_WARPS - 1): thread r holds weight row
     // tm * BM + r of the item; a warp reaches the TMEM lanes of its quarter
-    // and drains one quarter of the item's BN token columns.
-    const int q = warp & 3, r = q * 32 + (tid & 31);
+    // and drains one quarter of the item's BN token columns, 8 at a time.
+    // Each 32-row x 8-token block goes through shared memory so that lane l
+    // ends up with 8 consecutive weight rows (output columns) of one token:
+    // the functor then writes them as one 16-byte (bf16) or 32-byte (fp32)
+    // vector.
+    const int q = warp & 3, lane = tid & 31, r = q * 32 + lane;
     const int part = (warp - 2) / 4, c_lo = part * (BN / 4), c_hi = c_lo + BN / 4;
+    float* stg = epi_stage + (warp - 2) * (8 * EPI_PITCH);
+    const int tj = lane >> 2, rg = (lane & 3) * 8;  // token and first row this lane stores
     uint32_t li = 0;
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++li) {
       int bz, split, tm, tn;
@@ -182,12 +193,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (li >> 1) & 1, abort_flag, nullptr))) break;
       tc_fence_after();
       const uint32_t taddr = tbase + acc * BN + ((uint32_t)(q * 32) << 16);
-      const int col = tm * BM + r;
       float* pdst = nullptr;
       if (g.splits > 1)
         pdst = g.partial + (((long long)bz * per_z + tm * g.tiles_n + tn) * g.splits + split) * (long long)(BN * BM);
-      // Eight token columns at a time (a short body keeps the functor's code
-      // small enough for the instruction cache).
+      const int col0 = tm * BM + q * 32 + rg;  // first output column of this lane's 8
 #pragma unroll 1
       for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
         uint32_t v[8];
@@ -198,17 +207,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) v[j] = 0u;
         }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) stg[j * EPI_PITCH + lane] = __uint_as_float(v[j]);
+        __syncwarp();
+        float o[8];
+        {
+          const float4 a0 = *reinterpret_cast<const float4*>(stg + tj * EPI_PITCH + rg);
+          const float4 a1 = *reinterpret_cast<const float4*>(stg + tj * EPI_PITCH + rg + 4);
+          o[0] = a0.x; o[1] = a0.y; o[2] = a0.z; o[3] = a0.w;
+          o[4] = a1.x; o[5] = a1.y; o[6] = a1.z; o[7] = a1.w;
+        }
+        __syncwarp();  // the block is read before the next chunk overwrites it
+        const int tok = tn * BN + c0 + tj;
         if (pdst) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) __stcg(pdst + (c0 + j) * BM + r, __uint_as_float(v[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float mine = __uint_as_float(v[j]);
-            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            const int tok = tn * BN + c0 + j;
-            if ((r & 1) == 0 && col < g.Mw && tok < g.Nt) epi(bz, tok, col, mine, other);
-          }
+          float* d = pdst + (c0 + tj) * BM + q * 32 + rg;
+          reinterpret_cast<float4*>(d)[0] = make_float4(o[0], o[1], o[2], o[3]);
+          reinterpret_cast<float4*>(d)[1] = make_float4(o[4], o[5], o[6], o[7]);
+        } else if (col0 < g.Mw && tok < g.Nt) {
+          epi.store8(bz, tok, col0, o);
         }
       }
       tc_fence_before();

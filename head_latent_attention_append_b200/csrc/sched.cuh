@@ -117,7 +117,7 @@ __device__ __forceinline__ int find_le(const int* a, int n, int x) {
 // Row blocks whose tile offsets the schedule keeps in shared memory (the
 // binary searches below then cost no global round trips); beyond this they
 // stay in global memory.
-constexpr int kSchedSmemRb = 16384;
+constexpr int kSchedSmemRb = 49152;
 
 __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
   extern __shared__ int sched_smem[];
