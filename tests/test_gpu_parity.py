@@ -78,12 +78,13 @@ def test_prefill_matches_oracle_on_sampled_positions():
 
 
 # ------------------------------------------------------ small custom cases --
-def small_case(lengths, n_q, shuffle=True, dtype="bf16", spare=2, seed=5):
-    """A page_bf16_decode-shaped problem with the given cached lengths."""
+def small_case(lengths, n_q, shuffle=True, dtype="bf16", spare=2, seed=5, d_c=None, d_r=None):
+    """A page_bf16_decode-shaped problem with the given cached lengths
+    (optionally another latent width d_c or RoPE-key width d_r)."""
     mla, workload = _mods()
     base = synth.WORKLOADS["page_bf16_decode" if dtype == "bf16" else "tiny_fp32_decode"]
-    wl = synth.Workload("custom", 9, base.n_h, base.d_h, base.d_v, base.d_c, base.d_r, base.d_model, base.d_cq,
-                        dtype, "decode", len(lengths), n_q, 0)
+    wl = synth.Workload("custom", 9, base.n_h, base.d_h, base.d_v, d_c or base.d_c, d_r or base.d_r, base.d_model,
+                        base.d_cq, dtype, "decode", len(lengths), n_q, 0)
     dev = torch.device("cuda")
     dt = workload.TORCH_DTYPE[dtype]
     dims = workload.dims_of(wl)
@@ -131,6 +132,22 @@ def test_edge_lengths_match_oracle(n_q):
     for b in range(len(EDGE_LENGTHS)):
         ref = O.mla_decode(dims, w, c["H"][b], n_q)
         assert rel_err(out[b], ref) <= TOL["bf16"], (b, EDGE_LENGTHS[b])
+
+
+@pytest.mark.parametrize("d_c,d_r", [(256, 16), (256, 48), (128, 64)])
+def test_rope_share_and_latent_width_variants_match_oracle(d_c, d_r):
+    """The two CTAs split the RoPE-key columns 16 * (d_r / 32) : the rest, so
+    d_r = 16 leaves rank 0 without any and d_r = 48 gives the ranks 16 and 32
+    columns (boxes swizzled to 32 and 64 bytes in one launch); d_c = 128 gives
+    each CTA a single latent chunk."""
+    c = small_case([0, 1, 63, 64, 200, 700], 2, d_c=d_c, d_r=d_r)
+    out, _, e1, e2 = run_small(c)
+    assert e1 == 0 and e2 == 0
+    dims = oracle_dims(c["wl"])
+    w = O.Weights(**c["hw"].as_dict())
+    for b in range(6):
+        ref = O.mla_decode(dims, w, c["H"][b], 2)
+        assert rel_err(out[b], ref) <= TOL["bf16"], (d_c, d_r, b)
 
 
 def test_fp32_edge_lengths_match_oracle():
