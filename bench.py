@@ -119,11 +119,26 @@ def barrier(ws):
         dist.barrier()
 
 
+def kernel_code_hash(files) -> str:
+    """sha256 of the listed csrc files' code, concatenated in order, with
+    comments and whitespace removed (a comment edit does not change the
+    kernel)."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "head_latent_attention_append_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def measured_traffic(workload: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     capture (profiles/traffic.json), or None when there is none for this
-    workload or the kernel's sources changed since it was taken."""
-    import hashlib
+    workload or the kernel's code changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -131,11 +146,7 @@ def measured_traffic(workload: str):
         rec = json.load(fh).get(workload)
     if not rec:
         return None
-    h = hashlib.sha256()
-    for f in rec["source_files"]:
-        with open(os.path.join(ROOT, "head_latent_attention_append_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return rec["traffic_bytes"] if h.hexdigest() == rec["source_sha256"] else None
+    return rec["traffic_bytes"] if kernel_code_hash(rec["source_files"]) == rec["source_sha256"] else None
 
 
 PREFILL_SAMPLE_TOKENS = 1024   # causal prefix of one sequence per oracle prefill sample

@@ -23,12 +23,12 @@
 // steps and, for d_r = 32 or 64, equal (the score MMA is the longest tensor
 // job per page).  Each CTA streams only its own columns of every page (no byte
 // is read twice), computes the partial score over them (all of its Q slice is
-// the TMEM A operand), and sends the partial, rounded to bf16, to its peer through
-// distributed shared memory.  Both CTAs add the two bf16 partials in fp32 --
-// the same two numbers, so both see bit-identical scores and run identical
-// softmax state -- and each multiplies P (bf16, in TMEM) by its own latent
-// half.  TMEM columns: O [0, d_c/2), S [256, 320), Q slice [320, 480),
-// P [480, 512).
+// the TMEM A operand), and sends the partial, rounded to bf16, to its peer
+// through distributed shared memory.  Both CTAs add the two bf16 partials in
+// fp32 -- the same two numbers, so both see bit-identical scores and run
+// identical softmax state -- and each multiplies P (bf16, in TMEM) by its own
+// latent half.  TMEM columns: O [0, d_c/2), S [256, 320), the Q slice from 320
+// (at most 144 columns: 128 latent + 16 RoPE), P [480, 512).
 //
 // Shared memory (128-byte swizzled 64 x 64 chunks, loaded by TMA):
 //   score ring, 2 slots: this CTA's columns of a page (its latent chunks and
@@ -41,7 +41,9 @@
 //   four 16 KB exchange buffers, filled by the peer with bulk copies (one
 //     4 KB copy per sender warp per page, staged in a local 16 KB block) that
 //     complete on this CTA's mbarrier; four buffers make an overwrite of an
-//     unread one impossible (see XBUF).
+//     unread one impossible (see XBUF);
+//   two 1 KB slots of partial row maxima for the finishers' pair exchange
+//     (a segment's row sums borrow the idle one).
 // Segment metadata and page ids are loaded a step ahead so no global load
 // sits on a page's critical path.
 //

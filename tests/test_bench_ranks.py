@@ -64,12 +64,14 @@ def test_measured_traffic_follows_kernel_source(tmp_path, monkeypatch):
     csrc = tmp_path / "head_latent_attention_append_b200" / "csrc"
     csrc.mkdir(parents=True)
     (tmp_path / "profiles").mkdir()
-    (csrc / "k.cuh").write_bytes(b"kernel v1")
-    digest = hashlib.sha256(b"kernel v1").hexdigest()
+    (csrc / "k.cuh").write_text("int kernel_v1;  // first\n")
+    digest = hashlib.sha256(b"intkernel_v1;").hexdigest()  # code only: no comments, no whitespace
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
         {"wl": {"traffic_bytes": 1234, "source_files": ["k.cuh"], "source_sha256": digest}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.measured_traffic("wl") == 1234
     assert bench.measured_traffic("other") is None
-    (csrc / "k.cuh").write_bytes(b"kernel v2")
+    (csrc / "k.cuh").write_text("/* reworded */ int  kernel_v1;  // second\n")
+    assert bench.measured_traffic("wl") == 1234  # a comment edit is not a kernel change
+    (csrc / "k.cuh").write_text("int kernel_v2;\n")
     assert bench.measured_traffic("wl") is None
