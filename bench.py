@@ -198,6 +198,16 @@ def oracle_sample(name: str, k: int = 0):
             "tokens": nq, "what": what}
 
 
+def binding_roof(mode: str, n_q: int) -> str:
+    """The roof the attention kernel is held to.  A decode step with one new
+    token per sequence does 242 flop per cache byte (d_c = 512, d_r = 64),
+    about the ridge of the measured peaks, and is read as HBM-bound; with
+    n_q >= 2 new tokens per sequence every cache byte feeds n_q query tokens
+    (>= 484 flop per byte), and a causal prefill far more, so those are
+    tensor-bound."""
+    return "tensor" if mode == "prefill" or n_q >= 2 else "hbm"
+
+
 def metric_of(mode: str, nbytes: float, flops: float, seconds: float):
     """The workload's headline figure: latent-cache GB/s for decode, attention
     TFLOP/s for prefill."""
@@ -352,7 +362,8 @@ def run_ours(args):
     tc_roof = {"bound": "tensor", "achieved": tc_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                "frac": tc_tflops / tc_peak, "algorithmic_flops_per_launch": flops,
                "peak_kind": "bf16 sustained"}
-    main_roof, other_roof = (tc_roof, hbm_roof) if prefill else (hbm_roof, tc_roof)
+    main_roof, other_roof = ((tc_roof, hbm_roof) if binding_roof(wl.mode, wl.n_q) == "tensor"
+                             else (hbm_roof, tc_roof))
     roofline = dict(main_roof, traffic=measured_traffic(wl.name), kernel="latent attention (split-KV)",
                     peak_src=peaks["src"],
                     avg_kernel_ms=attn_avg_ms, streamed_cache_bytes_per_launch=streamed_bytes,

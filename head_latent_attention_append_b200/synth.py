@@ -62,6 +62,9 @@ WORKLOADS = {
         Workload("dsv2_bf16_prefill", 4, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "prefill", 4, 4096, 0),
         Workload("dsv2_ragged_decode", 5, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "decode", 128, 2, 0,
                  ragged=True, max_cached=32768),
+        # Multi-token (speculative-style) decode: 4 new tokens per sequence over ragged histories.
+        Workload("dsv2_spec4_decode", 6, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "decode", 64, 4, 0,
+                 ragged=True, max_cached=32768),
     ]
 }
 

@@ -75,3 +75,24 @@ def test_measured_traffic_follows_kernel_source(tmp_path, monkeypatch):
     assert bench.measured_traffic("wl") == 1234  # a comment edit is not a kernel change
     (csrc / "k.cuh").write_text("int kernel_v2;\n")
     assert bench.measured_traffic("wl") is None
+
+
+def test_binding_roof_follows_flops_per_cache_byte():
+    sys.path.insert(0, ROOT)
+    import bench
+    from head_latent_attention_append_b200 import synth
+    assert bench.binding_roof("decode", 1) == "hbm"
+    assert bench.binding_roof("decode", 2) == "tensor"
+    assert bench.binding_roof("prefill", 4096) == "tensor"
+    # Flops per unique cache byte of a decode step: every key feeds n_q query
+    # tokens (less the causal triangle of the new tokens themselves).
+    wl = synth.WORKLOADS["dsv2_bf16_decode"]
+    per_key = wl.n_h * (2 * wl.d_cr + 2 * wl.d_c)
+    assert abs(per_key / (wl.d_cr * 2) - 241.8) < 0.1
+    for name in ("dsv2_ragged_decode", "dsv2_spec4_decode"):
+        w = synth.WORKLOADS[name]
+        kv = synth.kv_lengths(w)
+        pairs = sum(int(L) - w.n_q + 1 + q for L in kv for q in range(w.n_q))
+        intensity = pairs * per_key / (int(kv.sum()) * w.d_cr * 2)
+        assert intensity >= 1.99 * 241.8, (name, intensity)
+        assert bench.binding_roof(w.mode, w.n_q) == "tensor"

@@ -47,7 +47,8 @@ def check_decode(s, tol):
 
 
 @pytest.mark.parametrize("name,count", [("tiny_fp32_decode", 1), ("page_bf16_decode", 8),
-                                        ("dsv2_bf16_decode", 4), ("dsv2_ragged_decode", 8)])
+                                        ("dsv2_bf16_decode", 4), ("dsv2_ragged_decode", 8),
+                                        ("dsv2_spec4_decode", 4)])
 def test_decode_matches_oracle(name, count):
     mla, workload = _mods()
     s = workload.setup(name, checked_count=count)
@@ -122,7 +123,7 @@ def run_small(c, page_table=None, cache_fill=0.0, cache=None):
 EDGE_LENGTHS = [0, 1, 62, 63, 64, 127, 128, 129, 1000]
 
 
-@pytest.mark.parametrize("n_q", [1, 2])
+@pytest.mark.parametrize("n_q", [1, 2, 3, 4, 8])
 def test_edge_lengths_match_oracle(n_q):
     c = small_case(EDGE_LENGTHS, n_q)
     out, _, e1, e2 = run_small(c)
@@ -183,28 +184,33 @@ def test_two_runs_are_bitwise_identical():
     np.testing.assert_array_equal(a, b)
 
 
-def test_later_new_token_does_not_reach_earlier_query():
+@pytest.mark.parametrize("n_q,j", [(2, 1), (4, 2)])
+def test_later_new_token_does_not_reach_earlier_query(n_q, j):
     mla, _ = _mods()
-    c = small_case([200, 64], 2)
+    c = small_case([200, 64], n_q)
     out, cache, _, _ = run_small(c)
-    # Overwrite the cache row of the second new token of sequence 0 and decode
-    # again without re-appending: query 0 must not change.
+    # Overwrite the cache row of new token j of sequence 0 and decode again
+    # without re-appending: the queries before j must not change, query j and
+    # the later ones must, and sequence 1 must not.
     wl, lay = c["wl"], c["lay"]
-    pos = int(c["kv"][0]) - 1
+    pos = int(c["kv"][0]) - n_q + j
     page = int(lay.page_table[0, pos // 64])
     cache2 = cache.clone()
     cache2[page, pos % 64] = 7.0
-    hq = torch.from_numpy(np.stack([c["H"][b][-2:] for b in range(2)])).to(c["dev"], c["dt"])
+    hq = torch.from_numpy(np.stack([c["H"][b][-n_q:] for b in range(2)])).to(c["dev"], c["dt"])
     out2 = torch.empty_like(torch.from_numpy(out)).to(c["dev"])
-    ws = torch.empty(mla.decode_workspace_bytes(c["dims"], 2, 2, int(c["kv"].max())), dtype=torch.uint8,
+    ws = torch.empty(mla.decode_workspace_bytes(c["dims"], 2, n_q, int(c["kv"].max())), dtype=torch.uint8,
                      device=c["dev"])
     pt = torch.from_numpy(lay.page_table).to(c["dev"])
     mla.decode(c["weights"], hq, torch.from_numpy(c["kv"]).to(c["dev"]), pt, lay.num_pages, cache2, out2,
                int(c["kv"].max()), ws)
     torch.cuda.synchronize()
     out2 = out2.cpu().numpy()
-    np.testing.assert_array_equal(out[0, 0], out2[0, 0])
-    assert not np.array_equal(out[0, 1], out2[0, 1])
+    for q in range(n_q):
+        if q < j:
+            np.testing.assert_array_equal(out[0, q], out2[0, q])
+        else:
+            assert not np.array_equal(out[0, q], out2[0, q]), q
     np.testing.assert_array_equal(out[1], out2[1])
 
 
