@@ -15,6 +15,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "cp.cuh"
 #include "gemm.cuh"
 #include "gemm_tc.cuh"
 #include "prep.cuh"
@@ -148,12 +149,15 @@ struct Plan {
       part_o, part_ml, obar, total;
   int R, qrows;
 };
-Plan make_plan(const mla_dims& d, int R, bool attention) {
+// cp: context-parallel partials, where every segment (at most W + R) has its
+// own partial slot.
+Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false) {
   const size_t e = esize(d);
   Plan P{};
   P.R = R;
   P.qrows = (d.dtype == MLA_BF16) ? 128 : d.n_h;
   const int W = kWorkerSlots;
+  const size_t slots = cp ? std::max<size_t>(2 * (size_t)W, (size_t)W + R) : 2 * (size_t)W;
   size_t o = 0;
   P.hdr = o;        o = align_up(o + 256, 256);
   P.counters = o;   o = align_up(o + sizeof(int) * kCounterCap, 256);
@@ -167,8 +171,8 @@ Plan make_plan(const mla_dims& d, int R, bool attention) {
     P.segs = o;       o = align_up(o + sizeof(Seg) * (size_t)(W + R), 256);
     P.rb_first = o;   o = align_up(o + sizeof(int) * (size_t)(R + 1), 256);
     P.split_rbs = o;  o = align_up(o + sizeof(int) * (size_t)(2 * W + 1), 256);
-    P.part_o = o;     o = align_up(o + sizeof(float) * (size_t)2 * W * d.n_h * d.d_c, 256);
-    P.part_ml = o;    o = align_up(o + sizeof(float) * (size_t)2 * W * d.n_h * 2, 256);
+    P.part_o = o;     o = align_up(o + sizeof(float) * slots * d.n_h * d.d_c, 256);
+    P.part_ml = o;    o = align_up(o + sizeof(float) * slots * d.n_h * 2, 256);
     P.obar = o;       o = align_up(o + e * (size_t)R * d.n_h * d.d_c, 256);
   }
   P.total = o;
@@ -368,11 +372,19 @@ mla_status append_impl(const mla_weights* w, const void* h, const int32_t* seq_i
                              ws, P, st));
 }
 
+// Context-parallel partial: the rank's window and where its (obar_r, lse_r)
+// go instead of the W_UV projection.
+struct CpOut {
+  CpWindow win;
+  void* obar;  // [R][n_h][d_c], type of the path
+  float* lse;  // [R][n_h]
+};
+
 template <typename T>
 mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_len, int uniform_kv_len,
                        int n_q, int prefill_S, const int32_t* page_table, int max_pages, int num_pages,
                        const void* cache, float* out, int R, int max_kv_len, void* ws, const Plan& P,
-                       cudaStream_t st) {
+                       cudaStream_t st, const CpOut* cp = nullptr) {
   const mla_dims& d = w->d;
   const int d_cr = d.d_c + d.d_r;
   const int din = d_in(d);
@@ -438,9 +450,13 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   {
     SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
     ++g_launches;
-    const size_t sched_smem = R + 1 <= kSchedSmemRb ? sizeof(int) * (size_t)(R + 1) : 0;
-    if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
-    sched_kernel<<<1, 1024, sched_smem, st>>>(sa);
+    if (cp) {
+      cp_sched_kernel<<<1, 1024, 0, st>>>(sa, cp->win);
+    } else {
+      const size_t sched_smem = R + 1 <= kSchedSmemRb ? sizeof(int) * (size_t)(R + 1) : 0;
+      if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
+      sched_kernel<<<1, 1024, sched_smem, st>>>(sa);
+    }
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (5) attention on the latent cache, (6) combine of split row blocks.
@@ -469,6 +485,11 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     kfn<<<dim3(W, G), attn_simt::THREADS, sm, st>>>(aa, HG);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
+  }
+  if (cp) {
+    ++g_launches;
+    cp_combine_kernel<T><<<dim3(R, ceil_div(d.n_h, 8)), 256, 0, st>>>(aa, static_cast<T*>(cp->obar), cp->lse);
+    return cuda_status(cudaGetLastError());
   }
   {
     ++g_launches;
@@ -663,6 +684,60 @@ mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_l
                                       B * n_q, max_kv_len, workspace, P, stream);
   return attend_impl<float>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out, B * n_q,
                             max_kv_len, workspace, P, stream);
+}
+
+size_t mla_decode_cp_workspace_bytes(const mla_dims* dims, int B, int n_q) {
+  if (check_dims(dims) != MLA_OK || dims->dtype != MLA_BF16 || B <= 0 || n_q <= 0) return 0;
+  return make_plan(*dims, B * n_q, true, true).total;
+}
+
+mla_status mla_decode_cp_partial(const mla_weights* w, const void* h_q, const int32_t* kv_len,
+                                 const int32_t* window_start, const int32_t* window_count,
+                                 const int32_t* page_table, int max_pages, int num_pages, const void* cache,
+                                 void* obar_out, float* lse_out, int B, int n_q, int max_kv_len, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || B <= 0 || n_q <= 0 || max_kv_len < n_q || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (w->d.dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if (!h_q || !kv_len || !window_start || !window_count || !page_table || !cache || !obar_out || !lse_out ||
+      !workspace)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h_q, 16) || !aligned(cache, 16) || !aligned(obar_out, 16) ||
+      !aligned(lse_out, 4))
+    return MLA_ERR_INVALID_ARG;
+  const Plan P = make_plan(w->d, B * n_q, true, true);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  CpOut cp{CpWindow{window_start, window_count, max_pages * w->d.page_size}, obar_out, lse_out};
+  return attend_impl<__nv_bfloat16>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, nullptr,
+                                    B * n_q, max_kv_len, workspace, P, stream, &cp);
+}
+
+mla_status mla_decode_cp_combine(const mla_weights* w, int n_ranks, const void* obar_parts,
+                                 const float* lse_parts, float* out, int B, int n_q, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || n_ranks <= 0 || B <= 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
+  if (w->d.dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if (!obar_parts || !lse_parts || !out || !workspace) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(obar_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16))
+    return MLA_ERR_INVALID_ARG;
+  const mla_dims& d = w->d;
+  const int R = B * n_q;
+  const Plan P = make_plan(d, R, true, true);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  using T = __nv_bfloat16;
+  ++g_launches;
+  cp_merge_kernel<T><<<dim3(R, ceil_div(d.n_h, 8)), 256, 0, stream>>>(
+      n_ranks, static_cast<const T*>(obar_parts), lse_parts, at<T>(workspace, P.obar), R, d.n_h, d.d_c,
+      at<int>(workspace, P.hdr));
+  cudaError_t e = cudaGetLastError();
+  if (e) return cuda_status(e);
+  EpiStore<float> epi{out, (long long)d.n_h * d.d_v, d.d_v, 1.f};
+  return cuda_status(gemm<T>(at<T>(workspace, P.obar), (long long)d.n_h * d.d_c, d.d_c, w->uv, d.d_c,
+                             (long long)d.d_v * d.d_c, R, d.d_v, d.d_c, d.n_h, epi, workspace, P, stream));
 }
 
 size_t mla_prefill_workspace_bytes(const mla_dims* dims, int B, int S) {

@@ -25,6 +25,7 @@ EXPORTED = [
     "mla_append_workspace_bytes", "mla_append_latent", "mla_decode_workspace_bytes", "mla_decode",
     "mla_prefill_workspace_bytes", "mla_prefill", "mla_get_error", "mla_status_string",
     "mla_last_launch_count", "mla_profile_begin", "mla_profile_end", "mla_append_latent_noalloc",
+    "mla_decode_cp_workspace_bytes", "mla_decode_cp_partial", "mla_decode_cp_combine",
 ]
 APPEND_NOALLOC_MAX_T = 256
 
@@ -70,6 +71,9 @@ def _load():
         "mla_profile_begin": (S, [I]),
         "mla_append_latent_noalloc": (S, [P, P, P, P, P, I, I, I, P, I, P, P]),
         "mla_profile_end": (S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
+        "mla_decode_cp_workspace_bytes": (Z, [D, I, I]),
+        "mla_decode_cp_partial": (S, [P, P, P, P, P, P, I, I, P, P, P, I, I, I, P, Z, P]),
+        "mla_decode_cp_combine": (S, [P, I, P, P, P, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -190,6 +194,28 @@ def prefill(w: Weights, h, page_table, num_pages: int, cache, out, workspace, st
     _check("mla_prefill", lib.mla_prefill(
         w.handle, _ptr(h), _ptr(page_table), page_table.shape[1], num_pages, _ptr(cache), _ptr(out), B, S,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_cp_workspace_bytes(dims: Dims, B: int, n_q: int) -> int:
+    return lib.mla_decode_cp_workspace_bytes(ctypes.byref(dims), B, n_q)
+
+
+def decode_cp_partial(w: Weights, h_q, kv_len, window_start, window_count, page_table, num_pages: int, cache,
+                      obar_out, lse_out, max_kv_len: int, workspace, stream=None):
+    """This rank's share of a context-parallel decode step (include/mla.h)."""
+    B, n_q = h_q.shape[0], h_q.shape[1]
+    _check("mla_decode_cp_partial", lib.mla_decode_cp_partial(
+        w.handle, _ptr(h_q), _ptr(kv_len), _ptr(window_start), _ptr(window_count), _ptr(page_table),
+        page_table.shape[1], num_pages, _ptr(cache), _ptr(obar_out), _ptr(lse_out), B, n_q, max_kv_len,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_cp_combine(w: Weights, obar_parts, lse_parts, out, workspace, stream=None):
+    """Merges all ranks' partials [n_ranks, B, n_q, ...] into out [B, n_q, n_h, d_v]."""
+    n_ranks, B, n_q = obar_parts.shape[0], obar_parts.shape[1], obar_parts.shape[2]
+    _check("mla_decode_cp_combine", lib.mla_decode_cp_combine(
+        w.handle, n_ranks, _ptr(obar_parts), _ptr(lse_parts), _ptr(out), B, n_q, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def get_error(workspace, stream=None) -> int:

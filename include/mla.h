@@ -176,6 +176,52 @@ mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_l
                       size_t workspace_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Context-parallel decode: one sequence's cache spread over several ranks
+ * (GPUs).  The pages do not split a sequence over devices; the split rests
+ * on the identity that the softmax denominators of disjoint key sets add up
+ * (the absorbed output of "ai-decoupled-rope-mla", absorption equations, is
+ * W_UV applied to a softmax-weighted latent sum, which merges exactly).
+ *
+ * Rank r holds one page-aligned window of each sequence b, positions
+ * window_start[b] .. window_start[b] + window_count[b] - 1 (device int32 [B];
+ * start a multiple of page_size; count 0 for none), in its own page pool:
+ * page_table [B, max_pages] maps the window's i-th page (positions
+ * start + i*page_size ..) to a page of `cache`.  Tokens are appended with
+ * mla_append_latent at their GLOBAL positions through a table indexed by
+ * global page (the window's pages at index start/page_size + i, -1 elsewhere),
+ * so the RoPE key carries the global position.
+ *
+ * mla_decode_cp_partial: for new token q of sequence b (global position
+ * kv_len[b]-n_q+q, kv_len the GLOBAL key count) and every head, the attention
+ * over the keys of the window at positions <= its own: writes the normalised
+ * latent sum obar_out [B, n_q, n_h, d_c] (bf16) and
+ * lse_out [B, n_q, n_h] (fp32) = log2 sum_t exp(a_t) over those keys; a row
+ * with no such key gets lse = -inf and an unspecified obar row.  A window that
+ * is negative, not page-aligned or longer than max_pages*page_size sets
+ * MLA_ERR_DEVICE_BOUNDS and counts as empty.
+ *
+ * mla_decode_cp_combine: merges every rank's partials, obar_parts
+ * [n_ranks, B, n_q, n_h, d_c] (bf16) and lse_parts [n_ranks, B, n_q, n_h]
+ * (fp32), as obar = sum_r 2^(lse_r - L) obar_r with L = log2 sum_r 2^lse_r,
+ * then writes out [B, n_q, n_h, d_v] (fp32) = W_UV,h obar_h.  A row that no
+ * rank saw sets MLA_ERR_DEVICE_BOUNDS and yields zeros.  The exchange of the
+ * partials between ranks (an all-gather) is the caller's.
+ *
+ * bf16 only (an fp32 mla_dims returns MLA_ERR_UNSUPPORTED).  Both calls take
+ * a workspace of mla_decode_cp_workspace_bytes(dims, B, n_q).
+ * ------------------------------------------------------------------------- */
+size_t mla_decode_cp_workspace_bytes(const mla_dims* dims, int B, int n_q);
+mla_status mla_decode_cp_partial(const mla_weights* w, const void* h_q, const int32_t* kv_len,
+                                 const int32_t* window_start, const int32_t* window_count,
+                                 const int32_t* page_table, int max_pages, int num_pages,
+                                 const void* cache, void* obar_out, float* lse_out, int B, int n_q,
+                                 int max_kv_len, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream);
+mla_status mla_decode_cp_combine(const mla_weights* w, int n_ranks, const void* obar_parts,
+                                 const float* lse_parts, float* out, int B, int n_q,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Causal prefill on the absorbed path.  h [B, S, d_model]: token s of
  * sequence b sits at position s.  Appends all B*S tokens to the cache (the
  * page table must cover S positions per sequence), then every token attends

@@ -28,6 +28,9 @@ section):
   The absorbed form (decoupled-RoPE page, "absorption saves cache" equations:
   ``q~ = W_UK^T q`` and ``W_UV sum_t alpha_t c_t``) is provided separately as a
   self-check, never as the oracle's answer.
+* Context-parallel decode (``window_partial``, ``merge_windows``,
+  ``latent_output``).  The pages do not split a sequence over devices; these
+  state the softmax-over-disjoint-key-sets identity a split relies on.
 * RoPE.  Pairs ``(2i, 2i+1)`` rotated by angle ``pos * theta_i`` with
   ``theta_i = base^(-2i/d_r)``; the pages print only the rotation family and its
   relative property ``R_m^T R_t = R_{t-m}`` ("ai-decoupled-rope-mla", decoupled
@@ -250,6 +253,73 @@ def mla_decode(dims: Dims, w: Weights, H: np.ndarray, n_q: int, **kw) -> np.ndar
     are the new queries (each appended to the cache before it attends)."""
     T = H.shape[0]
     return mla_sequence(dims, w, H, list(range(T - n_q, T)), **kw)
+
+
+# ----------------------------------------------------------------------------
+# Decode over a window of the keys (context-parallel split)
+# ----------------------------------------------------------------------------
+# The pages never split one sequence's keys across devices.  What such a split
+# needs is the plain identity for a softmax over a union of disjoint key sets:
+# with Z_j = sum over set j of exp(a_t), the full softmax-weighted latent sum is
+# sum_j (Z_j / sum_k Z_k) * (the softmax-weighted latent sum over set j).  The
+# functions below state it in base 2 (log2 Z_j), the form the library
+# exchanges between ranks.
+def window_partial(dims: Dims, w: Weights, H: np.ndarray, n_q: int, start: int, count: int,
+                   scale: Optional[float] = None):
+    """One window's share of a decode step of one sequence.
+
+    ``H`` [T, D] holds every token of the sequence; the last ``n_q`` are the
+    new queries at positions T-n_q .. T-1.  Keys are limited to positions
+    ``[start, start + count)`` and, per query, to positions <= its own.
+    Returns ``(o_bar [n_q, n_h, d_c], lse2 [n_q, n_h])``: the softmax-weighted
+    latent sum over those keys (scores against the latent with the absorbed
+    query ``q~ = W_UK,h^T q_C``) and ``log2 sum_t exp(a_t)``.  A query with no
+    such key gets ``o_bar = 0`` and ``lse2 = -inf``."""
+    w = as_f64(w)
+    H = np.asarray(H, dtype=np.float64)
+    T = H.shape[0]
+    n_h, d_h, d_c = dims.n_h, dims.d_h, dims.d_c
+    scale = dims.default_scale() if scale is None else scale
+    freqs = rope_frequencies(dims.d_r, dims.rope_base)
+    pos = np.arange(T, dtype=np.float64)
+    rows = np.arange(T - n_q, T)
+    keys = np.arange(max(0, start), min(T, start + count))
+    o_bar = np.zeros((n_q, n_h, d_c))
+    lse2 = np.full((n_q, n_h), -np.inf)
+    if keys.size == 0:
+        return o_bar, lse2
+    c, k_r = cache_entries(w, H[keys], pos[keys], freqs)
+    q_c, q_r = queries(w, dims, H[rows], pos[rows], freqs)
+    q_abs = np.einsum("qhd,hdc->qhc", q_c, w.W_UK.reshape(n_h, d_h, d_c))
+    a = (np.einsum("qhc,tc->qht", q_abs, c) + np.einsum("qhr,tr->qht", q_r, k_r)) * scale
+    visible = keys[None, :] <= rows[:, None]                      # [Q, K]
+    for qi in range(n_q):
+        if not visible[qi].any():
+            continue
+        aq = a[qi][:, visible[qi]]                                 # [n_h, K']
+        m = aq.max(axis=1, keepdims=True)
+        e = np.exp(aq - m)
+        z = e.sum(axis=1)
+        o_bar[qi] = (e @ c[visible[qi]]) / z[:, None]
+        lse2[qi] = (m[:, 0] + np.log(z)) / math.log(2.0)
+    return o_bar, lse2
+
+
+def merge_windows(parts):
+    """Merges window partials ``[(o_bar_j, lse2_j), ...]`` of the same queries
+    into the latent sum over the union of the windows: weights
+    ``2^(lse2_j - L)`` with ``L = log2 sum_j 2^lse2_j`` (windows with
+    ``lse2 = -inf`` weigh nothing)."""
+    lse = np.stack([p[1] for p in parts])                         # [J, Q, n_h]
+    L = np.log2(np.sum(np.exp2(lse - lse.max(axis=0)), axis=0)) + lse.max(axis=0)
+    wts = np.exp2(lse - L)                                        # [J, Q, n_h]
+    return sum(wts[j][..., None] * parts[j][0] for j in range(len(parts)))
+
+
+def latent_output(dims: Dims, w: Weights, o_bar: np.ndarray) -> np.ndarray:
+    """``o_h = W_UV,h o_bar_h`` for o_bar [Q, n_h, d_c]; returns [Q, n_h, d_v]."""
+    W_UV = np.asarray(w.W_UV, np.float64).reshape(dims.n_h, dims.d_v, dims.d_c)
+    return np.einsum("qhc,hvc->qhv", np.asarray(o_bar, np.float64), W_UV)
 
 
 # ----------------------------------------------------------------------------

@@ -52,6 +52,12 @@ def test_size_queries(mla):
     assert mla.absorbed_weights_bytes(dims3(mla, n_h=0)) == 0
     assert mla.decode_workspace_bytes(d, 0, 1, 10) == 0
     assert mla.decode_workspace_bytes(d, 4, 2, 1) == 0
+    # Context-parallel partials: one partial slot per segment (more row blocks
+    # than the decode path's slots need a larger workspace); bf16 only.
+    assert mla.decode_cp_workspace_bytes(d, 64, 1) >= mla.decode_workspace_bytes(d, 64, 1, 8193)
+    assert mla.decode_cp_workspace_bytes(d, 1024, 1) > mla.decode_workspace_bytes(d, 1024, 1, 8193)
+    assert mla.decode_cp_workspace_bytes(dims3(mla, dtype=mla.F32), 4, 1) == 0
+    assert mla.decode_cp_workspace_bytes(d, 0, 1) == 0
 
 
 def test_status_strings(mla):
@@ -87,6 +93,9 @@ def test_bad_arguments_are_rejected_before_launch(mla):
     assert lib.mla_decode(None, FAKE, FAKE, FAKE, 4, 4, FAKE, FAKE, 1, 1, 10, FAKE, 1 << 30, None) == -1
     assert lib.mla_append_latent(None, FAKE, FAKE, FAKE, FAKE, 1, 4, 4, FAKE, 1, FAKE, 1 << 30, None) == -1
     assert lib.mla_prefill(None, FAKE, FAKE, 4, 4, FAKE, FAKE, 1, 8, FAKE, 1 << 30, None) == -1
+    assert lib.mla_decode_cp_partial(None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, FAKE, FAKE, FAKE, 1, 1, 10, FAKE,
+                                     1 << 30, None) == -1
+    assert lib.mla_decode_cp_combine(None, 2, FAKE, FAKE, FAKE, 1, 1, FAKE, 1 << 30, None) == -1
     assert lib.mla_get_error(None, None) == -1
     assert lib.mla_weights_dims(None, ctypes.byref(d)) == -1
 
