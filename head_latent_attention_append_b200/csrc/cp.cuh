@@ -121,7 +121,8 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 // normalised latent sum obar_r (type T) and lse_r = m + log2 l.  A row block
 // without a segment gets lse_r = -inf and its obar_r row is left unwritten.
 // Block = (row block, 8 heads), one warp per head; lane j holds latent
-// columns 4j .. 4j+3 of each 128-column chunk (d_c <= 512, d_c % 64 == 0).
+// columns 4j .. 4j+3 of each 128-column chunk (the bf16 path has d_c <= 512,
+// d_c % 128 == 0).
 template <typename T>
 __global__ void __launch_bounds__(256) cp_combine_kernel(AttnArgs a, T* obar_out, float* lse_out) {
   const Sched& S = a.sched;

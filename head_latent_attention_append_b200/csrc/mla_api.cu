@@ -4,6 +4,7 @@
 // stream.
 #include "../../include/mla.h"
 
+#include <limits.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -709,7 +710,8 @@ mla_status mla_decode_cp_partial(const mla_weights* w, const void* h_q, const in
   if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
   mla_status s = begin_call(workspace, stream, P);
   if (s != MLA_OK) return s;
-  CpOut cp{CpWindow{window_start, window_count, max_pages * w->d.page_size}, obar_out, lse_out};
+  const int max_count = (int)std::min<long long>((long long)max_pages * w->d.page_size, INT_MAX);
+  CpOut cp{CpWindow{window_start, window_count, max_count}, obar_out, lse_out};
   return attend_impl<__nv_bfloat16>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, nullptr,
                                     B * n_q, max_kv_len, workspace, P, stream, &cp);
 }
