@@ -145,3 +145,70 @@ def test_exchange_on_two_gloo_ranks():
     for rank, err, own in res:
         assert own is True, (rank, own)
         assert err <= 1e-12, (rank, err)
+
+
+def _orchestration_worker(rank, ws, port, q):
+    """cp.decode_cp on one gloo rank, with libmla's two calls stood in for by
+    the oracle (test-only fakes): checks the step's buffers, the exchange
+    and the hand-off to the merge."""
+    sys.path.insert(0, ROOT)
+    import types
+    import oracle as Ow
+    from head_latent_attention_append_b200 import cp as cpw
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        wl, dims, w = _small(0)
+        n_q, lengths = 2, [150, 40, 1]
+        kv = np.asarray(lengths, np.int32) + n_q
+        H = [synth.make_hidden(wl, b, int(kv[b])) for b in range(len(lengths))]
+        win = cpw.shard_windows(kv, ws, 16)[rank]
+
+        def fake_partial(wt, h_q, kv_len, start, count, pt, num_pages, cache, obar_out, lse_out, max_kv_len,
+                         workspace, stream=None):
+            for b in range(h_q.shape[0]):
+                o, ls = Ow.window_partial(dims, w, H[b], n_q, int(start[b]), int(count[b]))
+                obar_out[b] = torch.from_numpy(o)
+                lse_out[b] = torch.from_numpy(ls)
+
+        def fake_combine(wt, obar_parts, lse_parts, out, workspace, stream=None):
+            for b in range(out.shape[0]):
+                parts = [(obar_parts[r, b].numpy(), lse_parts[r, b].double().numpy())
+                         for r in range(obar_parts.shape[0])]
+                out[b] = torch.from_numpy(Ow.latent_output(dims, w, Ow.merge_windows(parts)))
+
+        fake_mla = types.SimpleNamespace(decode_cp_partial=fake_partial, decode_cp_combine=fake_combine)
+        import head_latent_attention_append_b200 as pkg
+        sys.modules["head_latent_attention_append_b200.mla"] = fake_mla
+        pkg.mla = fake_mla
+        h_q = torch.from_numpy(np.stack([H[b][-n_q:] for b in range(len(lengths))]).astype(np.float64))
+        out = torch.empty((len(lengths), n_q, dims.n_h, dims.d_v), dtype=torch.float64)
+        wts = types.SimpleNamespace(dims=dims)
+        obar_parts, lse_parts = cpw.decode_cp(wts, h_q, torch.from_numpy(kv), torch.from_numpy(win.start),
+                                              torch.from_numpy(win.count), None, 0, None, out, int(kv.max()), None)
+        err = max(float(np.abs(out[b].numpy() - Ow.mla_decode(dims, w, H[b], n_q)).max()
+                        / np.abs(Ow.mla_decode(dims, w, H[b], n_q)).max()) for b in range(len(lengths)))
+        q.put((rank, err, tuple(obar_parts.shape), tuple(lse_parts.shape)))
+        dist.barrier()
+    except Exception as e:  # report instead of leaving the parent waiting
+        q.put((rank, float("inf"), repr(e), None))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_decode_step_orchestration_on_three_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ws = 3
+    procs = [ctx.Process(target=_orchestration_worker, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for rank, err, oshape, lshape in res:
+        assert err <= 1e-6, (rank, err, oshape)   # lse travels as fp32
+        assert oshape == (ws, 3, 2, 4, 16) and lshape == (ws, 3, 2, 4), (oshape, lshape)
