@@ -20,6 +20,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -76,6 +77,93 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+# Clock-event reason bits (NVML): name in the JSON line, NVML constant suffix, value.
+NVML_REASONS = (("hw_slowdown", "HwSlowdown", 0x8), ("hw_thermal_slowdown", "HwThermalSlowdown", 0x40),
+                ("sw_thermal_slowdown", "SwThermalSlowdown", 0x20), ("sw_power_cap", "SwPowerCap", 0x4))
+
+
+def summarize_nvml(samples, max_mhz):
+    """(sm_mhz, reason bitmask) samples -> the line's clocks object, or None."""
+    if not samples:
+        return None
+    seen = 0
+    for _, bits in samples:
+        seen |= bits
+    return {"sm_mhz": statistics.median(m for m, _ in samples), "sm_max_mhz": max_mhz,
+            "reasons": sorted(name for name, _, bit in NVML_REASONS if seen & bit), "samples": len(samples),
+            "source": "NVML, every 2 ms during the timed region"}
+
+
+class NvmlPoller:
+    """Reads the SM clock and the clock-event reasons through NVML (read-only)
+    from a host thread every ~2 ms while a timed region runs: the regions
+    here last milliseconds, well under nvidia-smi's 200 ms period.  Any NVML
+    failure leaves it without samples; it never raises."""
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.dev = device_index
+        self.period = period_s
+        self.nv = None
+        self.h = None
+        self.max_mhz = None
+        self.samples = []
+        self.thread = None
+        self.stop_evt = threading.Event()
+
+    def _handle(self, nv):
+        import torch
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            pass
+        try:
+            return nv.nvmlDeviceGetHandleByPciBusId(
+                "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id))
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def start(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = self._handle(nv)
+            self.reasons = (getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                            or nv.nvmlDeviceGetCurrentClocksThrottleReasons)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self._shutdown()
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                                     int(self.reasons(self.h))))
+            except Exception:
+                return
+            self.stop_evt.wait(self.period)
+
+    def _shutdown(self):
+        if self.nv is not None:
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+            self.nv = None
+
+    def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=2.0)
+        self._shutdown()
+        return summarize_nvml(list(self.samples), self.max_mhz)
 
 
 def dist_setup():
@@ -315,15 +403,21 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    poller = NvmlPoller(local)
+    poller.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    in_region = poller.stop()
     barrier(ws)
     ms_step, value = aggregate(units, e0.elapsed_time(e1) / args.steps, ws, scale=scale)
-    clk = clocks.stop()
+    smi = clocks.stop()
+    # The NVML samples inside the timed region when there are any; the
+    # nvidia-smi samples around it otherwise (and alongside, for reference).
+    clk = dict(in_region, nvidia_smi=smi) if in_region else smi
     assert mla.get_error(s.ws) == mla.MLA_OK
 
     # End to end through the public API with host buffers: pinned h_new in,

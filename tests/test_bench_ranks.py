@@ -96,3 +96,37 @@ def test_binding_roof_follows_flops_per_cache_byte():
         intensity = pairs * per_key / (int(kv.sum()) * w.d_cr * 2)
         assert intensity >= 1.99 * 241.8, (name, intensity)
         assert bench.binding_roof(w.mode, w.n_q) == "tensor"
+
+
+def test_nvml_poller_summarises_in_region_samples(monkeypatch):
+    """The clock poller against a fake NVML (no GPU here): samples taken on a
+    thread, reasons OR-ed over the samples, and a broken NVML yields None."""
+    import types
+    import time as _time
+    sys.path.insert(0, ROOT)
+    import bench
+    clocks = iter([1965.0, 1965.0, 1800.0] * 1000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1, nvmlInit=lambda: None, nvmlShutdown=lambda: None,
+        nvmlDeviceGetHandleByUUID=lambda u: "h", nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setattr(torch.cuda, "get_device_properties",
+                        lambda i: types.SimpleNamespace(uuid="abc", pci_domain_id=0, pci_bus_id=1, pci_device_id=0))
+    p = bench.NvmlPoller(0, period_s=0.001)
+    p.start()
+    _time.sleep(0.05)
+    out = p.stop()
+    assert out["samples"] >= 3 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["sm_mhz"] in (1965.0, 1800.0)
+    assert bench.summarize_nvml([(1900.0, 0x8 | 0x40), (1950.0, 0)], 1965) == {
+        "sm_mhz": 1925.0, "sm_max_mhz": 1965, "reasons": ["hw_slowdown", "hw_thermal_slowdown"], "samples": 2,
+        "source": "NVML, every 2 ms during the timed region"}
+    # NVML that fails to start leaves no samples and raises nothing.
+    broken = types.SimpleNamespace(nvmlInit=lambda: (_ for _ in ()).throw(RuntimeError("no driver")),
+                                   nvmlShutdown=lambda: None)
+    monkeypatch.setitem(sys.modules, "pynvml", broken)
+    q = bench.NvmlPoller(0)
+    q.start()
+    assert q.stop() is None
