@@ -109,3 +109,10 @@ def test_handle_arguments_checked_before_launch(mla):
     # workspace instead.
     d = dims3(mla)
     assert mla.decode_workspace_bytes(d, 2, 1, 100) > 4096
+
+
+def test_binding_fails_loudly_without_the_library(mla, monkeypatch, tmp_path):
+    """No fallback: with libmla.so absent the binding refuses to load."""
+    monkeypatch.setattr(mla, "LIB_PATH", str(tmp_path / "libmla.so"))
+    with pytest.raises(ImportError, match="libmla.so not built"):
+        mla._load()
