@@ -28,10 +28,18 @@ struct AttnArgs {
   int uniform_kv_len, n_q, max_kv_len;
   Sched sched;
   float* part_o;             // [2W][n_h][d_c]
-  float* part_ml;            // [2W][n_h][2]
+  float* part_ml;            // [2W][2][n_h][2]: (m, l) per latent-column half (ml_index)
   void* obar;                // [R][n_h][d_c] (type of the path)
   int* err;
 };
+
+// Index into part_ml of the (m, l) pair of partial slot `slot`, latent-column
+// half `half` ([0, d_c/2) or [d_c/2, d_c)) and head h.  The tensor-core
+// kernel's two CTAs each keep their own softmax state for their half; the
+// CUDA-core kernel writes the same pair to both halves.
+__host__ __device__ __forceinline__ long long ml_index(int slot, int half, int n_h, int h) {
+  return (((long long)slot * 2 + half) * n_h + h) * 2;
+}
 
 namespace attn_simt {
 constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
@@ -154,8 +162,11 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
         for (int r = 0; r < MAX_CPT; ++r)
           if (r < cpt && oj + r * TPH < a.d_c) po[oj + r * TPH] = o[r];
         if (oj == 0) {
-          a.part_ml[((long long)g.slot * a.n_h + h) * 2 + 0] = m;
-          a.part_ml[((long long)g.slot * a.n_h + h) * 2 + 1] = l;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            a.part_ml[ml_index(g.slot, half, a.n_h, h) + 0] = m;
+            a.part_ml[ml_index(g.slot, half, a.n_h, h) + 1] = l;
+          }
         }
       }
     }
@@ -192,19 +203,28 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (h >= a.n_h) return;
   const int s0 = S.rb_seg_first[rb], s1 = S.rb_seg_first[rb + 1];
-  // Row max and sum over the segments.
-  float m = -INFINITY;
-  for (int s = s0 + lane; s < s1; s += 32) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
+  // Row max and sum over the segments, for each latent-column half.
+  float m[2] = {-INFINITY, -INFINITY};
+  for (int s = s0 + lane; s < s1; s += 32)
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float l = 0.f;
-  for (int s = s0 + lane; s < s1; s += 32) {
-    const float* ml = a.part_ml + ((long long)S.segs[s].slot * a.n_h + h) * 2;
-    l += exp2f(ml[0] - m) * ml[1];
-  }
+    for (int hf = 0; hf < 2; ++hf) m[hf] = fmaxf(m[hf], a.part_ml[ml_index(S.segs[s].slot, hf, a.n_h, h)]);
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  const float inv = 1.f / l;
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m[hf] = fmaxf(m[hf], __shfl_xor_sync(0xffffffffu, m[hf], o));
+  float l[2] = {0.f, 0.f};
+  for (int s = s0 + lane; s < s1; s += 32)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const float* ml = a.part_ml + ml_index(S.segs[s].slot, hf, a.n_h, h);
+      l[hf] += exp2f(ml[0] - m[hf]) * ml[1];
+    }
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], o);
+  const float inv[2] = {1.f / l[0], 1.f / l[1]};
+  const int half_cols = a.d_c / 2;
   T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
   // All four 128-column chunks (d_c <= 512) at once, so a warp's loads are in
   // flight together.
@@ -212,17 +232,19 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int sb = s0; sb < s1; sb += 32) {
-    // Lane k holds segment sb + k's slot and weight; broadcast in order.
+    // Lane k holds segment sb + k's slot and weights; broadcast in order.
     int slot = 0;
-    float wgt = 0.f;
+    float wgt0 = 0.f, wgt1 = 0.f;
     if (sb + lane < s1) {
       slot = S.segs[sb + lane].slot;
-      wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
+      wgt0 = exp2f(a.part_ml[ml_index(slot, 0, a.n_h, h)] - m[0]);
+      wgt1 = exp2f(a.part_ml[ml_index(slot, 1, a.n_h, h)] - m[1]);
     }
     const int cnt = min(32, s1 - sb);
     for (int k = 0; k < cnt; ++k) {
       const int sl = __shfl_sync(0xffffffffu, slot, k);
-      const float w = __shfl_sync(0xffffffffu, wgt, k);
+      const float w0 = __shfl_sync(0xffffffffu, wgt0, k);
+      const float w1 = __shfl_sync(0xffffffffu, wgt1, k);
       const float* src = a.part_o + ((long long)sl * a.n_h + h) * a.d_c;
       float4 v[4];
 #pragma unroll
@@ -232,6 +254,7 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        const float w = (c * 128 + 4 * lane) < half_cols ? w0 : w1;
         acc[c].x += w * v[c].x;
         acc[c].y += w * v[c].y;
         acc[c].z += w * v[c].z;
@@ -242,7 +265,8 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const int j = c * 128 + 4 * lane;
-    if (j < a.d_c) store4(out + j, acc[c].x * inv, acc[c].y * inv, acc[c].z * inv, acc[c].w * inv);
+    const float iv = j < half_cols ? inv[0] : inv[1];
+    if (j < a.d_c) store4(out + j, acc[c].x * iv, acc[c].y * iv, acc[c].z * iv, acc[c].w * iv);
   }
 }
 

@@ -20,42 +20,59 @@
 //   rank 0: latent columns [0, d_c/2) and the first ra RoPE-key columns
 //   rank 1: latent columns [d_c/2, d_c) and the other rb = d_r - ra,
 // with ra = 16 * (d_r / 32) so that both score shares are whole 16-column MMA
-// steps and, for d_r = 32 or 64, equal (the score MMA is the longest tensor
-// job per page).  Each CTA streams only its own columns of every page (no byte
-// is read twice), computes the partial score over them (all of its Q slice is
-// the TMEM A operand), and sends the partial, rounded to bf16, to its peer
-// through distributed shared memory.  Both CTAs add the two bf16 partials in
-// fp32 -- the same two numbers, so both see bit-identical scores and run
-// identical softmax state -- and each multiplies P (bf16, in TMEM) by its own
-// latent half.  TMEM columns: O [0, d_c/2), S [256, 320), the Q slice from 320
-// (at most 144 columns: 128 latent + 16 RoPE), P [480, 512).
+// steps and, for d_r = 32 or 64, equal.  Each CTA streams only its own
+// columns of every page (no byte is read twice from HBM) and computes the
+// partial score over them into TMEM.  The partial goes to the peer as fp16
+// (saturated at +-65504, log2 units) through distributed shared memory, in
+// the 128-byte-swizzled K-major layout a tensor-core operand has, and each
+// CTA's tensor core adds the peer's partial to its own with one more MMA
+// against a 64 x 64 identity matrix: S = S_own + X_peer * I, exact in the
+// fp32 accumulator.  So the softmax threads read finished fp32 scores from
+// TMEM and do no conversion work.  Each CTA keeps its own exact partial, so
+// the two CTAs' scores differ by the rounding of one fp16 partial and each
+// runs its own softmax state (m, l) for its half of the latent columns: each
+// half is normalised by its own state, and split row blocks leave one
+// (m, l) per half.  fp16's 11-bit significand keeps this well below the
+// rounding the bf16 cache rows put into every score (a bf16 exchange doubled
+// the error against the fp64 oracle once logits reach ~30).
 //
-// Shared memory (128-byte swizzled 64 x 64 chunks, loaded by TMA):
+// TMEM columns: O [0, d_c/2), two score buffers S0 [256, 320) and
+// S1 [320, 384), the latent part of this CTA's Q slice from 384 (at most 128
+// columns).  A score buffer is free again as soon as the finishers have read
+// it; P (bf16) goes to a shared-memory tile that the SS P*V MMA reads.
+//
+// Shared memory (1024-byte aligned pieces):
+//   three 16 KB exchange buffers, written by the peer's sender threads with
+//     asynchronous remote stores (st.async, 16 bytes each, straight from
+//     registers) that complete on this CTA's mbarrier; the MMA that consumes
+//     one returns it to the peer with a tcgen05.commit multicast onto the
+//     peer's credit barrier.  (A staged bulk copy goes through the TMA engine
+//     behind the page loads and landed ~1.6 us after issue; the remote
+//     stores skip that queue.);
 //   score ring, 2 slots: this CTA's columns of a page (its latent chunks and
 //     its RoPE share, loaded with a 16- or 32-column box swizzled to 32 or 64
 //     bytes), freed as soon as the page's score MMA completes;
 //   latent ring, 2 slots: the page's latent columns again (4 chunks) for
 //     P*V, freed by P*V.  The second read is an L2 hit (the first was a few
-//     microseconds earlier), so HBM still sees every byte once; decoupling
-//     the rings keeps a page's HBM load off the softmax's critical loop;
-//   four 16 KB exchange buffers, filled by the peer with bulk copies (one
-//     4 KB copy per sender warp per page, staged in a local 16 KB block) that
-//     complete on this CTA's mbarrier; four buffers make an overwrite of an
-//     unread one impossible (see XBUF);
-//   two 1 KB slots of partial row maxima for the finishers' pair exchange
+//     microseconds earlier), so HBM still sees every byte once;
+//   the RoPE part of the Q slice (SS MMA operand, swizzled like the page's
+//     RoPE share), the fp16 identity matrix, and the 16 KB P tile;
+//   two 1 KB slots of half-row maxima for the finishers' pair exchange
 //     (a segment's row sums borrow the idle one).
 // Segment metadata and page ids are loaded a step ahead so no global load
 // sits on a page's critical path.
 //
 // Warp roles (512 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
 // allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
-// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-7 =
-// sender (reads each page's partial score, ships it to the peer, loads Q),
-// warps 8-11 and 12-15 = the two finisher halves (keys 0-31 and 32-63 of
-// every row: combine, softmax, P, and half of O in the epilogue); thread r of
-// any of these owns row r = TMEM lane r.  The sender runs a page ahead of the
-// finishers, so the exchange of one page overlaps the softmax of the previous
-// one.  Every wait is bounded (sm100::mbar_wait).
+// exchange-MMA and P*V-MMA issuer (it polls the inputs of both streams and
+// issues whichever is ready, so neither waits on the other), all
+// warp-uniform with one elected lane issuing; warps 4-7 = sender (reads each page's own partial score from TMEM,
+// ships it to the peer, loads each segment's Q slice), warps 8-11 and 12-15 =
+// the two finisher halves (keys 0-31 and 32-63 of every row: softmax, P, and
+// half of O in the epilogue); thread r of any of these owns row r = TMEM
+// lane r.  Two score buffers let the score MMA of page t+1 run while the
+// finishers work on page t.  Every wait is bounded (sm100::mbar_wait; warp
+// 3's poll loop gives up after 2^32 cycles without progress).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -71,31 +88,32 @@ constexpr int MAX_PV = 4;                     // latent chunks per CTA per page 
 constexpr int MAX_ROPE = 32;                  // RoPE-key columns per CTA (d_r <= 64)
 constexpr int SGROUPS = 2;                    // score ring: a page's own columns, freed by its score MMA
 constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
-constexpr int XBUF = 4;                       // exchange buffers per CTA
-// No partial can overwrite one that is still unread, with no extra barrier:
-// each finisher half reads the peer's partial of page t before it takes its
-// own page t + 1 out of the staging block, which the sender needs (from both
-// halves) before it ships page t + 2.  The peer's finishers wait for that
-// page t + 2 before they take their page t + 3 out of staging, which the
-// peer's sender needs before it ships page t + 4 into the buffer page t used.
-static_assert(XBUF >= 4, "the exchange needs four buffers (see above)");
+constexpr int XBUF = 3;                       // exchange buffers per CTA (credit-controlled)
 constexpr int ROPE_OFF = MAX_PV * CHUNK_BYTES;  // a score slot: latent chunks, then the RoPE share
 constexpr int SG_BYTES = ROPE_OFF + KT * MAX_ROPE * 2;
 constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
-constexpr int X_BYTES = 128 * KT * 2;         // one bf16 partial-score tile
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_P = 480, TM_COLS = 512;
+constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
+constexpr int QR_BYTES = 128 * MAX_ROPE * 2;  // the RoPE part of the Q slice
+constexpr int ID_BYTES = KT * KT * 2;         // 64 x 64 fp16 identity
+constexpr int P_BYTES = 128 * KT * 2;         // P tile: 128 rows x 64 keys bf16
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384, TM_COLS = 512;
 
-// The exchange buffers and their barriers sit at the same offsets in both
-// CTAs (the peer addresses them through mapa).
+// The exchange buffers and the credit barriers sit at the same offsets in
+// both CTAs (the peer addresses them through mapa / a commit multicast).
 constexpr int OFF_X = 0;
-constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
-constexpr int OFF_SG = OFF_XS + X_BYTES;
+constexpr int OFF_SG = OFF_X + XBUF * X_BYTES;
 constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
-constexpr int OFF_MH = OFF_VG + VGROUPS * VG_BYTES;  // half-row maxima [2][2][128] fp32 (sums reuse a slot)
+constexpr int OFF_QR = OFF_VG + VGROUPS * VG_BYTES;
+constexpr int OFF_ID = OFF_QR + QR_BYTES;
+constexpr int OFF_P = OFF_ID + ID_BYTES;
+constexpr int OFF_MH = OFF_P + P_BYTES;           // half-row maxima [2][2][128] fp32 (sums reuse a slot)
 constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * SGROUPS + 2 * VGROUPS + XBUF + 9 + 4;
+constexpr int NUM_BARS = 2 * XBUF + 2 * SGROUPS + 2 * VGROUPS + 2 + 2 + 2 + 2 + 1 + 1 + 3 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
+static_assert(OFF_SG % 1024 == 0 && OFF_VG % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_ID % 1024 == 0 &&
+                  OFF_P % 1024 == 0 && SG_BYTES % 1024 == 0,
+              "swizzled operands need 1024-byte aligned tiles");
 // No slack for aligning the base: the kernel has no static shared memory, so
 // its dynamic block starts on a 1024-byte boundary (the kernel checks this
 // and reports MLA_ERR_UNSUPPORTED otherwise).
@@ -137,42 +155,54 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
-// a peer CTA's, completing as transaction bytes on the peer's mbarrier
-// `bar_cluster_addr`.  One copy carries what would otherwise be many small
-// remote stores, each with its own transaction-count update at the peer.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster_addr, uint32_t src_smem, uint32_t bytes,
-                                                  uint32_t bar_cluster_addr) {
+// Asynchronous 16-byte store into a peer CTA's shared memory that completes
+// as 16 transaction bytes on the peer's mbarrier `bar_cluster_addr`.
+__device__ __forceinline__ void st_async_peer(uint32_t dst_cluster_addr, uint4 v, uint32_t bar_cluster_addr) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
           dst_cluster_addr),
-      "r"(src_smem), "r"(bytes), "r"(bar_cluster_addr)
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
       : "memory");
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Asks L2 to fetch `bytes` (a multiple of 16) from global memory ahead of use.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
-// Waits until the sources of this thread's committed bulk copies have been read.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Partial scores travel between the CTAs as bf16 pairs: packing is one
-// conversion, unpacking is two integer ops (no conversion-pipe work).
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
+// Arrives once on the mbarrier at the same shared-memory offset in every CTA
+// of `cta_mask` when every tcgen05 operation this thread issued has completed.
+__device__ __forceinline__ void tc_commit_to(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+// Partial scores travel between the CTAs as fp16 pairs, saturated at
+// +-65504 (one conversion per pair).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t u;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
+  return u;
+}
+// Instruction descriptor, kind::f16 with fp16 A and B (the exchanged
+// partials against the identity), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Byte offset, in an exchange tile, of 16-byte piece u (0..7) of row r's 64
-// bf16 partial scores.  Layout [row][128 bytes], so each warp's 32 rows form
-// one contiguous 4 KB block (one bulk copy); the pieces are XOR-swizzled by
-// the row so that the eight rows a quarter-warp touches at once fall in
-// eight different bank groups.
-constexpr int X_WARP_BYTES = 32 * KT * 2;
+// Byte offset, in an exchange tile (and in the P tile), of 16-byte piece u
+// (0..7) of row r's 64 16-bit values: row r at r * 128, piece u at
+// (u ^ (r & 7)) * 16.  This is the 128-byte-swizzled K-major operand layout
+// (8-row groups of 1 KB), so a received tile is the A operand of the exchange
+// MMA as it lands, and the eight rows a quarter-warp writes at once fall in
+// eight bank groups.
 __device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+// Byte offset of 16-byte piece u of row r in the RoPE part of the Q slice,
+// rows of rw * 2 bytes swizzled to that width (64-byte rows: piece ^ row
+// bits 1-2; 32-byte rows: piece ^ row bit 2), matching sdesc_swz.
+__device__ __forceinline__ uint32_t qr_off(int r, int u, int rw) {
+  return rw == 32 ? (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) : (uint32_t)(r * 32 + ((u ^ ((r >> 2) & 1)) << 4));
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap rmap16,
@@ -184,20 +214,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
-  uint64_t* sg_full = x_full + XBUF;     // [SGROUPS]
+  uint64_t* x_free = x_full + XBUF;      // [XBUF] the peer has consumed what this CTA sent into its buffer
+  uint64_t* sg_full = x_free + XBUF;     // [SGROUPS]
   uint64_t* sg_empty = sg_full + SGROUPS;
   uint64_t* vg_full = sg_empty + SGROUPS;  // [VGROUPS]
   uint64_t* vg_empty = vg_full + VGROUPS;
-  uint64_t* s_full = vg_empty + VGROUPS;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* pv_done = s_full + 3;
-  uint64_t* q_ready = s_full + 4;
-  uint64_t* o_free = s_full + 5;
-  uint64_t* final_bar = s_full + 6;
-  uint64_t* xs_full = s_full + 7;  // the sender has staged a page's partial
-  uint64_t* xs_free = s_full + 8;  // the finishers have taken it out of the staging block
-  uint64_t* pair_bars = s_full + 9;  // [4]: the two finisher warps of a lane quarter
+  uint64_t* s_full = vg_empty + VGROUPS;   // [2] own partial score in buffer b
+  uint64_t* s_read = s_full + 2;           // [2] the sender has read the own partial in buffer b
+  uint64_t* s_total = s_read + 2;          // [2] the peer's partial has been added into buffer b
+  uint64_t* s_free = s_total + 2;          // [2] the finishers have read buffer b
+  uint64_t* p_ready = s_free + 2;          // P of the current page is in the P tile
+  uint64_t* pv_done = p_ready + 1;         // P*V of the current page has completed
+  uint64_t* q_ready = pv_done + 1;
+  uint64_t* o_free = q_ready + 1;
+  uint64_t* final_bar = q_ready + 2;
+  uint64_t* pair_bars = q_ready + 3;       // [4]: the two finisher warps of a lane quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -210,10 +241,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int rw = rank ? p.rb : p.ra;               // RoPE-key columns this CTA scores (0, 16 or 32)
   const int rx = a.d_c + (rank ? p.ra : 0);        // and the first of them
   const CUtensorMap* rmap = rw == 32 ? &rmap32 : &rmap16;
+  const uint64_t rswz = rw == 32 ? kSwizzle64 : kSwizzle32;
   const Seg* segs = a.sched.segs;
   const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
   if (tid == 32) {
+    for (int i = 0; i < XBUF; ++i) {
+      mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
+      mbar_init(&x_free[i], 1);  // the peer's commit
+    }
     for (int i = 0; i < SGROUPS; ++i) {
       mbar_init(&sg_full[i], 1);
       mbar_init(&sg_empty[i], 1);
@@ -222,19 +258,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&vg_full[i], 1);
       mbar_init(&vg_empty[i], 1);
     }
-    for (int i = 0; i < XBUF; ++i) mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);   // sender
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_read[i], 128);  // sender
+      mbar_init(&s_total[i], 1);
+      mbar_init(&s_free[i], 256);  // finishers
+    }
     mbar_init(p_ready, 256);  // finishers
     mbar_init(pv_done, 1);
     mbar_init(q_ready, 128);  // sender
     mbar_init(o_free, 256);   // finishers
     mbar_init(final_bar, 2);  // one commit per issuer warp
-    mbar_init(xs_full, 128);
-    mbar_init(xs_free, 256);
     for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
     *abort_flag = 0;
     mbar_fence_init();
+  }
+  // The 64 x 64 fp16 identity (B operand of the exchange MMA), K-major with
+  // the 128-byte swizzle: row n holds 1.0 at column n.
+  {
+    const int n = tid >> 3, u = tid & 7;  // 512 threads: one 16-byte piece each
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if ((n >> 3) == u) {
+      uint32_t* e = reinterpret_cast<uint32_t*>(&v);
+      e[(n & 7) >> 1] = (n & 1) ? 0x3C000000u : 0x00003C00u;
+    }
+    *reinterpret_cast<uint4*>(smem + OFF_ID + n * 128 + ((u ^ (n & 7)) << 4)) = v;
     fence_proxy_async_smem();
   }
   if (warp == 2) {
@@ -307,74 +355,130 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mbar_wait_warp(&full[q], (last / nring) & 1, abort_flag, nullptr, 50000000ull, false);
       }
     }
-  } else if (warp == 1 || warp == 3) {
-    // ------------------------------------------------------ MMA issuers
-    // Warp 1 issues the partial-score MMAs, warp 3 the P*V MMAs; each blocks
-    // only on its own inputs, and each tcgen05.commit tracks only the MMAs
-    // its own thread issued.
-    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q, tP = tbase + TM_P;
-    const uint32_t sSG = smem_u32(smem + OFF_SG), sVG = smem_u32(smem + OFF_VG);
+  } else if (warp == 1) {
+    // ------------------------------------------------- score-MMA issuer
+    // Page t's partial score goes into buffer t & 1, free once the finishers
+    // have read page t - 2's scores from it.
+    const uint32_t tS = tbase + TM_S, tQ = tbase + TM_Q;
+    const uint32_t sSG = smem_u32(smem + OFF_SG), sQR = smem_u32(smem + OFF_QR);
+    const uint32_t idS = idesc_bf16(128, 64, 0, 0);
     uint32_t tg = 0, seg_k = 0;
     bool ok = true;
-    if (warp == 1) {
-      const uint32_t idS = idesc_bf16(128, 64, 0, 0);
-      Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-      for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const Seg g = gn;
-        if (si + 1 < seg_hi) gn = segs[si + 1];  // in flight while this segment runs
-        const int n = g.t_hi - g.t_lo;
-        if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
+    Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
+    for (int si = seg_lo; si < seg_hi && ok; ++si) {
+      const Seg g = gn;
+      if (si + 1 < seg_hi) gn = segs[si + 1];  // in flight while this segment runs
+      const int n = g.t_hi - g.t_lo;
+      if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
+      tc_fence_after();
+      for (int i = 0; i < n; ++i, ++tg) {
+        const uint32_t b = tg & 1;
+        if (tg >= 2 && !(ok = mbar_wait_warp(&s_free[b], ((tg - 2) >> 1) & 1, abort_flag, a.err))) break;
+        const uint32_t gs = tg % SGROUPS;
+        if (!(ok = mbar_wait_warp(&sg_full[gs], (tg / SGROUPS) & 1, abort_flag, a.err))) break;
         tc_fence_after();
-        for (int i = 0; i < n; ++i) {
-          if (tg > 0 && !(ok = mbar_wait_warp(s_free, (tg - 1) & 1, abort_flag, a.err))) break;
-          const uint32_t gs = tg % SGROUPS;
-          if (!(ok = mbar_wait_warp(&sg_full[gs], (tg / SGROUPS) & 1, abort_flag, a.err))) break;
+        if (elect_one()) {
+          const uint32_t gb = sSG + gs * SG_BYTES, d = tS + b * KT;
+          for (int q = 0; q < npv; ++q) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_ts(d, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
+                     (q | k) ? 1u : 0u);
+          }
+          // The RoPE share: rows of rw * 2 bytes, swizzled to that width, both
+          // operands in shared memory.
+          for (int k = 0; k < rw / 16; ++k)
+            mma_ss(d, sdesc_swz(sQR + k * 32, 8 * rw * 2, rswz), sdesc_swz(gb + ROPE_OFF + k * 32, 8 * rw * 2, rswz),
+                   idS, 1u);
+          tc_commit(&s_full[b]);
+          tc_commit(&sg_empty[gs]);  // the score ring slot is free once its MMAs are done
+        }
+        __syncwarp();
+      }
+      ++seg_k;
+    }
+    if (elect_one()) tc_commit(final_bar);
+    __syncwarp();
+    mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
+  } else if (warp == 3) {
+    // ---------------------------------------- exchange-MMA and P*V issuer
+    // Two in-order streams: the exchange MMA of page t (S_t += X_peer,t * I,
+    // once the sender has read the own partial and the peer's has landed;
+    // its completion also hands the exchange buffer back to the peer) and
+    // P*V of page t (once the finishers have written P_t).  The warp polls
+    // the inputs of both and issues whichever is ready, so a late peer copy
+    // never holds back P*V and the reverse.
+    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O;
+    const uint32_t sX = smem_u32(smem + OFF_X), sID = smem_u32(smem + OFF_ID), sVG = smem_u32(smem + OFF_VG);
+    const uint32_t sP = smem_u32(smem + OFF_P);
+    const uint32_t idX = idesc_f16(128, KT), idPV = idesc_bf16(128, dh, 0, 1);
+    int total = 0;  // pages of this worker
+    for (int s = seg_lo + (tid & 31); s < seg_hi; s += 32) total += segs[s].t_hi - segs[s].t_lo;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    uint32_t xt = 0, pt = 0;       // next page of each stream
+    int si = seg_lo, pi = 0, seg_k = 0;  // P*V stream: segment, page in it, segment count
+    int seg_n = seg_lo < seg_hi ? segs[seg_lo].t_hi - segs[seg_lo].t_lo : 0;
+    // Progress deadline in SM cycles (clock64 is a register read; the global
+    // timer is far slower to read, which would delay every poll): 2^32 cycles,
+    // 2-4 s at the clocks this part runs at.
+    long long t_prog = clock64();
+    while ((int)pt < total) {
+      bool prog = false;
+      if ((int)xt < total) {
+        const uint32_t b = xt & 1, xb = xt % XBUF;
+        if (mbar_try_wait_warp(&s_read[b], (xt >> 1) & 1) && mbar_try_wait_warp(&x_full[xb], (xt / XBUF) & 1)) {
+          fence_proxy_async_smem();  // the peer's stores, now visible here, to the MMA's proxy
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t gb = sSG + gs * SG_BYTES;
-            for (int q = 0; q < npv; ++q) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_ts(tS, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
-                       (q | k) ? 1u : 0u);
-            }
-            // The RoPE share: rows of rw * 2 bytes, swizzled to that width.
-            for (int k = 0; k < rw / 16; ++k)
-              mma_ts(tS, tQ + npv * 32 + k * 8,
-                     sdesc_swz(gb + ROPE_OFF + k * 32, 8 * rw * 2, rw == 32 ? kSwizzle64 : kSwizzle32), idS, 1u);
-            tc_commit(s_full);
-            tc_commit(&sg_empty[gs]);  // the score ring slot is free once its MMAs are done
+            for (int k = 0; k < KT / 16; ++k)
+              mma_ss(tS + b * KT, sdesc_sw128(sX + xb * X_BYTES + k * 32, 16, 1024),
+                     sdesc_sw128(sID + k * 32, 16, 1024), idX, 1u);
+            tc_commit(&s_total[b]);
+            tc_commit_to(&x_free[xb], (uint16_t)(1u << peer));  // the peer may refill buffer xb
           }
           __syncwarp();
-          ++tg;
+          ++xt;
+          prog = true;
         }
-        ++seg_k;
       }
-    } else {
-      const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
-      Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-      for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const Seg g = gn;
-        if (si + 1 < seg_hi) gn = segs[si + 1];
-        const int n = g.t_hi - g.t_lo;
-        for (int i = 0; i < n; ++i) {
-          if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
-          if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
-          const uint32_t vs = tg % VGROUPS;
-          if (!(ok = mbar_wait_warp(&vg_full[vs], (tg / VGROUPS) & 1, abort_flag, a.err))) break;
+      if (pt < xt) {
+        const uint32_t vs = pt % VGROUPS;
+        if (mbar_try_wait_warp(p_ready, pt & 1) &&
+            (pi != 0 || seg_k == 0 || mbar_try_wait_warp(o_free, (seg_k - 1) & 1)) &&
+            mbar_try_wait_warp(&vg_full[vs], (pt / VGROUPS) & 1)) {
           tc_fence_after();
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < KT / 16; ++kk)
-              mma_ts(tO, tP + kk * 8, sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
-                     (i == 0 && kk == 0) ? 0u : 1u);
+              mma_ss(tO, sdesc_sw128(sP + kk * 32, 16, 1024),
+                     sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
+                     (pi == 0 && kk == 0) ? 0u : 1u);
             tc_commit(pv_done);
             tc_commit(&vg_empty[vs]);
           }
           __syncwarp();
-          ++tg;
+          ++pt;
+          if (++pi == seg_n) {
+            pi = 0;
+            ++seg_k;
+            if (++si < seg_hi) seg_n = segs[si].t_hi - segs[si].t_lo;
+          }
+          prog = true;
         }
-        ++seg_k;
+      }
+      if (prog) {
+        t_prog = clock64();
+      } else if (*abort_flag) {
+        break;
+      } else if (clock64() - t_prog > (1ll << 32)) {
+        if (elect_one()) {
+          *abort_flag = 1;
+          flag_error(a.err, kErrTimeout);
+        }
+        __syncwarp();
+        break;
       }
     }
     if (elect_one()) tc_commit(final_bar);
@@ -383,22 +487,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp >= 4) {
     // ------------------------------------------- sender and finisher warpgroups
     // Thread r of either warpgroup owns row r (= TMEM lane r) of the page.
-    // The sender (warps 4-7) reads each page's partial score (all 64 keys),
-    // packs it to bf16, stages it and ships it to the peer with one bulk copy
-    // per warp; it also loads each segment's Q slice.  The finisher (warps
-    // 8-11) owns whole rows: it adds its own staged partial to the peer's,
-    // keeps the running max and sum, writes P and runs the segment epilogue.
-    // The two work on consecutive pages at once, so the exchange of page t+1
-    // overlaps the softmax of page t, and no row is split between threads.
     const bool sender = warp < 8;
     const int h = warp >= 12 ? 1 : 0;  // finisher half: keys [32h, 32h + 32)
     const int r = tid - (sender ? 128 : 256 + 128 * h);
     const int lane = tid & 31;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O;
-    const uint32_t tQ = tbase + lane_off + TM_Q, tP = tbase + lane_off + TM_P + 16 * h;
-    uint8_t* sX = smem + OFF_X;
-    uint8_t* sXS = smem + OFF_XS;
+    const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O, tQ = tbase + lane_off + TM_Q;
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
@@ -406,10 +500,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
 
     if (sender) {
-      const uint32_t peer_x = map_peer(smem_u32(sX), peer);
+      // Reads each page's own partial score (all 64 keys of its row) from
+      // TMEM, packs it to fp16 and stores it straight into the peer's
+      // exchange buffer; also loads each segment's Q slice.
+      uint8_t* sQR = smem + OFF_QR;
+      const uint32_t peer_x = map_peer(smem_u32(smem + OFF_X), peer);
       const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
       const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
-      // Row r of this CTA's Q slice (chunks c_lo .. c_lo + n_own - 1) into TMEM.
+      // Row r of this CTA's Q slice: the latent chunks c_lo .. c_lo + npv - 1
+      // into TMEM, the RoPE share into shared memory.
       auto load_q = [&](int rb) {
         const uint4* src =
             (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
@@ -425,41 +524,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           tmem_st32(tQ + q * 32, wv);
         }
-        if (rw) {
-          uint32_t wv[16];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 v = (src && u * 8 < rw) ? __ldg(src + (rx + u * 8) / 8) : make_uint4(0, 0, 0, 0);
-            wv[4 * u + 0] = v.x;
-            wv[4 * u + 1] = v.y;
-            wv[4 * u + 2] = v.z;
-            wv[4 * u + 3] = v.w;
-          }
-          if (rw == 32) {
-            tmem_st16(tQ + npv * 32, wv);
-          } else {
-            uint32_t w8[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) w8[j] = wv[j];
-            tmem_st8(tQ + npv * 32, w8);
-          }
+        for (int u = 0; u < rw / 8; ++u) {
+          const uint4 v = src ? __ldg(src + (rx + u * 8) / 8) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(sQR + qr_off(r, u, rw)) = v;
         }
+        fence_proxy_async_smem();  // the MMA (async proxy) reads what the threads wrote
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(q_ready);
       };
       // Segment metadata stays in registers, the next segment's loaded a
       // segment ahead.
+      Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
       Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : Seg{};
-      int n_cur = 0;
-      if (seg_lo < seg_hi) {
-        const Seg g0 = segs[seg_lo];
-        load_q(g0.rb);
-        n_cur = g0.t_hi - g0.t_lo;
-      }
+      if (seg_lo < seg_hi) load_q(g_cur.rb);
       // The next segment's query rows are pulled into L2 while this segment
-      // streams, so loading them at the segment boundary reads L2, not HBM
-      // (prefill, with a boundary every ~32 pages, gains about 3%).
+      // streams, so loading them at the segment boundary reads L2, not HBM.
       const uint32_t q_half = (uint32_t)((a.n_h + 1) / 2) * a.d_cr * 2;
       auto prefetch_q = [&](int rb) {
         if (tid == 128) {
@@ -470,50 +550,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       };
       uint32_t tg = 0;
       for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const int n = n_cur;
+        const Seg g = g_cur;
+        const int n = g.t_hi - g.t_lo;
         if (si + 1 < seg_hi) prefetch_q(g_nxt.rb);
         for (int i = 0; i < n; ++i, ++tg) {
-          const uint32_t xb = tg % XBUF;
-          if (!(ok = wait_all(s_full, tg & 1))) break;
+          const uint32_t b = tg & 1, xb = tg % XBUF;
+          if (!(ok = wait_all(&s_full[b], (tg >> 1) & 1))) break;
           tc_fence_after();
           uint32_t cur[32];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t v[32];
-            tmem_ld32(tS + 32 * half, v);
+            tmem_ld32(tS + b * KT + 32 * half, v);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              cur[16 * half + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+              cur[16 * half + j] = pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          }
+          // Keys past the row block's end (the tail of its last page) may hold
+          // anything, NaN included; the peer's exchange MMA multiplies every
+          // key of a row by the identity's zeros too, so they travel as 0.
+          const int valid_all = min(KT, g.nkeys - (g.t_lo + i) * KT);
+          if (valid_all < KT) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              if (2 * x >= valid_all) cur[x] = 0u;
+              else if (2 * x + 1 >= valid_all) cur[x] &= 0x0000ffffu;
+            }
           }
           tc_fence_before();
-          mbar_arrive(s_free);
-          // The staging block is reused: the finisher must have taken the
-          // previous page out of it, and the copy engine must have read it.
-          if (lane == 0) bulk_wait_read_all();
-          if (tg > 0 && !(ok = wait_all(xs_free, (tg - 1) & 1))) break;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(sXS + x_off(r, u)) =
-                make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]);
-          fence_proxy_async_smem();  // the copy engine reads what the threads wrote
-          __syncwarp();
-          if (lane == 0) {
-            const uint32_t blk = (uint32_t)((warp & 3) * X_WARP_BYTES);
-            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, X_WARP_BYTES, peer_xbar + xb * 8);
-            bulk_commit();
-          }
-          // The peer's partial of this page will land in exchange buffer xb.
-          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
-          mbar_arrive(xs_full);
+          mbar_arrive(&s_read[b]);
           // The segment's scores are all read after its last page, so the next
           // segment's Q may replace this one's.
           if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
+          // The peer's partial of this page will land in exchange buffer xb.
+          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
+          // Buffer xb of the peer is free once its exchange MMA of page
+          // tg - XBUF has completed.
+          if (tg >= XBUF && !(ok = wait_all(&x_free[xb], ((tg / XBUF) - 1) & 1))) break;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            st_async_peer(peer_x + xb * X_BYTES + x_off(r, u),
+                          make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]), peer_xbar + xb * 8);
         }
-        n_cur = g_nxt.t_hi - g_nxt.t_lo;
+        g_cur = g_nxt;
         if (si + 2 < seg_hi) g_nxt = segs[si + 2];
       }
-      if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
+      // Every credit the peer returns lands before this CTA may exit: wait for
+      // its consumption of the last pages shipped (page p is the (p / XBUF)-th
+      // use of buffer p % XBUF).
+      if (ok)
+        for (uint32_t pg = tg > (uint32_t)XBUF ? tg - XBUF : 0; pg < tg; ++pg)
+          if (!wait_all(&x_free[pg % XBUF], (pg / XBUF) & 1)) break;
     } else {
       // Two finisher warpgroups: half h owns keys [32h, 32h + 32) of every
       // row and half of O's columns; the two threads of a row (their warps
@@ -532,6 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
       Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
       uint8_t* sV = smem + OFF_VG;
+      uint8_t* sPt = smem + OFF_P;
       float m_used = -INFINITY, l = 0.f;
       uint32_t tg = 0;
       for (int si = seg_lo; si < seg_hi && ok; ++si) {
@@ -539,34 +628,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int n = g.t_hi - g.t_lo;
         for (int i = 0; i < n; ++i, ++tg) {
           const int t = g.t_lo + i;
-          const uint32_t xb = tg % XBUF;
-          // This CTA's partial, staged by the sender; the block goes straight
-          // back to it.
-          if (!(ok = wait_all(xs_full, tg & 1))) break;
-          uint4 own4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) own4[u] = *reinterpret_cast<const uint4*>(sXS + x_off(r, 4 * h + u));
-          mbar_arrive(xs_free);
-          // The peer's partial: its bulk copy completes this CTA's barrier,
-          // and the phase completing makes the copied bytes visible here.
-          if (!(ok = wait_all(&x_full[xb], (tg / XBUF) & 1))) break;
+          const uint32_t b = tg & 1;
+          // Own + peer partial, summed by the exchange MMA.
+          if (!(ok = wait_all(&s_total[b], (tg >> 1) & 1))) break;
+          tc_fence_after();
           float s[32];
           {
-            const uint8_t* src = sX + xb * X_BYTES;
+            uint32_t v[32];
+            tmem_ld32(tS + b * KT + 32 * h, v);
+            tmem_ld_wait();
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint4 pv = *reinterpret_cast<const uint4*>(src + x_off(r, 4 * h + u));
-              const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-              const uint32_t mw[4] = {own4[u].x, own4[u].y, own4[u].z, own4[u].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 x = unpack_bf16x2(mw[e]);
-                const float2 y = unpack_bf16x2(pw[e]);
-                s[8 * u + 2 * e] = x.x + y.x;
-                s[8 * u + 2 * e + 1] = x.y + y.y;
-              }
-            }
+            for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
           }
+          tc_fence_before();
+          mbar_arrive(&s_free[b]);  // the score MMA of page tg + 2 may overwrite it
           const int valid_all = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
           const int valid = valid_all - 32 * h;             // valid keys among this half's 32
           if (valid < 32) {
@@ -616,7 +691,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
             psum = ps[0];
           }
-          // The previous P*V must be done before P is overwritten or O rescaled.
+          // The previous page's P*V must be done before P is overwritten or O
+          // rescaled.
           if (tg > 0) {
             if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
             tc_fence_after();
@@ -632,8 +708,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             l *= scale;
           }
-          tmem_st16(tP, pk);
-          tmem_st_wait();
+          // P row r, keys 32h .. 32h + 31: pieces 4h .. 4h + 3 of the
+          // 128-byte-swizzled K-major tile (the SS P*V MMA's A operand).
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(sPt + x_off(r, 4 * h + u)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
           l += psum;
           if (valid_all < KT) {
             // Keys past the end: P is 0 there, but 0 * NaN would still poison
@@ -647,8 +727,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0, 0, 0, 0);
             }
-            fence_proxy_async_smem();
           }
+          fence_proxy_async_smem();  // the MMA (async proxy) reads P and the cleared rows
           tc_fence_before();
           mbar_arrive(p_ready);
           if (i + 1 < n) continue;
@@ -666,7 +746,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const float lrow = ls[r] + ls[128 + r];
           if (!(ok = pair_sync())) break;
           // A whole row block is normalised into obar (bf16); a piece of a
-          // split row block leaves its unnormalised sum and (m, l) in its slot.
+          // split row block leaves its unnormalised sum and this CTA's (m, l)
+          // in its slot.
           const bool whole = g.slot < 0;
           const float inv = 1.f / lrow;
           for (int cc = hc0; cc < hc1; ++cc) {
@@ -695,9 +776,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               }
             }
           }
-          if (!whole && rank == 0 && h == 0 && r < a.n_h) {
-            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 0] = m_used;
-            a.part_ml[((long long)g.slot * a.n_h + r) * 2 + 1] = lrow;
+          if (!whole && h == 0 && r < a.n_h) {
+            float* ml = a.part_ml + ml_index(g.slot, (int)rank, a.n_h, r);
+            ml[0] = m_used;
+            ml[1] = lrow;
           }
           tc_fence_before();
           mbar_arrive(o_free);

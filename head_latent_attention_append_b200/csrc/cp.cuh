@@ -135,29 +135,43 @@ __global__ void __launch_bounds__(256) cp_combine_kernel(AttnArgs a, T* obar_out
     if (lane == 0) lse_out[row] = -INFINITY;
     return;
   }
-  float m = -INFINITY;
-  for (int s = s0 + lane; s < s1; s += 32) m = fmaxf(m, a.part_ml[((long long)S.segs[s].slot * a.n_h + h) * 2]);
+  // Max and sum over the segments, for each latent-column half (the two CTAs
+  // of the tensor-core kernel keep their own softmax state, equal to within
+  // the fp16 rounding of the exchanged partial scores).
+  float m[2] = {-INFINITY, -INFINITY};
+  for (int s = s0 + lane; s < s1; s += 32)
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float l = 0.f;
-  for (int s = s0 + lane; s < s1; s += 32) {
-    const float* ml = a.part_ml + ((long long)S.segs[s].slot * a.n_h + h) * 2;
-    l += exp2f(ml[0] - m) * ml[1];
-  }
+    for (int hf = 0; hf < 2; ++hf) m[hf] = fmaxf(m[hf], a.part_ml[ml_index(S.segs[s].slot, hf, a.n_h, h)]);
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m[hf] = fmaxf(m[hf], __shfl_xor_sync(0xffffffffu, m[hf], o));
+  float l[2] = {0.f, 0.f};
+  for (int s = s0 + lane; s < s1; s += 32)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const float* ml = a.part_ml + ml_index(S.segs[s].slot, hf, a.n_h, h);
+      l[hf] += exp2f(ml[0] - m[hf]) * ml[1];
+    }
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], o);
+  const int half_cols = a.d_c / 2;
   float4 acc[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = s0; s < s1; ++s) {
     const int slot = S.segs[s].slot;
-    const float wgt = exp2f(a.part_ml[((long long)slot * a.n_h + h) * 2] - m);
+    const float w0 = exp2f(a.part_ml[ml_index(slot, 0, a.n_h, h)] - m[0]);
+    const float w1 = exp2f(a.part_ml[ml_index(slot, 1, a.n_h, h)] - m[1]);
     const float* src = a.part_o + ((long long)slot * a.n_h + h) * a.d_c;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int j = c * 128 + 4 * lane;
       if (j < a.d_c) {
         const float4 v = load4(src + j);
+        const float wgt = j < half_cols ? w0 : w1;
         acc[c].x += wgt * v.x;
         acc[c].y += wgt * v.y;
         acc[c].z += wgt * v.z;
@@ -165,14 +179,17 @@ __global__ void __launch_bounds__(256) cp_combine_kernel(AttnArgs a, T* obar_out
       }
     }
   }
-  const float inv = 1.f / l;
+  const float inv[2] = {1.f / l[0], 1.f / l[1]};
   T* out = obar_out + row * a.d_c;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const int j = c * 128 + 4 * lane;
-    if (j < a.d_c) store4(out + j, acc[c].x * inv, acc[c].y * inv, acc[c].z * inv, acc[c].w * inv);
+    const float iv = j < half_cols ? inv[0] : inv[1];
+    if (j < a.d_c) store4(out + j, acc[c].x * iv, acc[c].y * iv, acc[c].z * iv, acc[c].w * iv);
   }
-  if (lane == 0) lse_out[row] = m + log2f(l);
+  // One log-sum-exp per row: the first half's (the second half's differs by
+  // the rounding of the exchanged scores).
+  if (lane == 0) lse_out[row] = m[0] + log2f(l[0]);
 }
 
 // Merges the ranks' partials of every (row, head) into obar (type T):

@@ -60,6 +60,7 @@ struct EpiAppend {
   double theta[32];        // RoPE frequencies
   int max_pages, num_pages, page_size, d_c, d_cr, n_seq;
   int* err;
+  OutT* dense;             // optional: every row also at dense[m * d_cr] (token order), else null
   __device__ void operator()(int, int m, int n, float v0, float v1) const {
     int s, p;
     if (seq_idx) {
@@ -80,6 +81,7 @@ struct EpiAppend {
     }
     if (n >= d_c) rope_rotate_pair(v0, v1, p, theta[(n - d_c) >> 1]);
     store_pair(cache + ((long long)page * page_size + p % page_size) * d_cr + n, v0, v1);
+    if (dense) store_pair(dense + (long long)m * d_cr + n, v0, v1);
   }
   // Columns n0 .. n0 + 7 of token m (n0 a multiple of 8; d_c is one too, so
   // the eight are all latent or all position key).
@@ -109,6 +111,7 @@ struct EpiAppend {
       for (int i = 0; i < 4; ++i) rope_rotate_pair(w[2 * i], w[2 * i + 1], p, theta[((n0 - d_c) >> 1) + i]);
     }
     mla::store8(cache + ((long long)page * page_size + p % page_size) * d_cr + n0, w);
+    if (dense) mla::store8(dense + (long long)m * d_cr + n0, w);
   }
 };
 
@@ -158,6 +161,53 @@ struct EpiQProj {
       w[2 * i + 1] = qr_scale * x1;
     }
     mla::store8(qabs + ((long long)m * qabs_rows + h) * d_cr + d_c + jj, w);
+  }
+};
+
+// Query projection for the materialised form: q = [q_C | RoPE_m(q_R)] per
+// head, both parts multiplied by qscale (the softmax scale times log2 e),
+// written to q[t][h][0 .. d_h + d_r).  Columns [0, n_h*d_h) are q_C (head h
+// at h*d_h), the rest q_R (head h at n_h*d_h + h*d_r).  Token m of a prefill
+// is position m % prefill_S.
+template <typename OutT>
+struct EpiQProjM {
+  OutT* q;                 // [T, n_h, d_h + d_r]
+  double theta[32];
+  int n_h, d_h, d_r, prefill_S;
+  float qscale;
+  __device__ void operator()(int, int m, int n, float v0, float v1) const {
+    const int nc = n_h * d_h, dq = d_h + d_r;
+    if (n < nc) {
+      const int h = n / d_h, i = n - h * d_h;
+      store_pair(q + ((long long)m * n_h + h) * dq + i, qscale * v0, qscale * v1);
+      return;
+    }
+    const int j = n - nc, h = j / d_r, jj = j - h * d_r;
+    rope_rotate_pair(v0, v1, m % prefill_S, theta[jj >> 1]);
+    store_pair(q + ((long long)m * n_h + h) * dq + d_h + jj, qscale * v0, qscale * v1);
+  }
+  // Columns n0 .. n0 + 7 (n0 a multiple of 8; d_h and d_r are too, so the
+  // eight belong to one head's q_C or one head's q_R).
+  __device__ void store8(int, int m, int n0, const float (&v)[8]) const {
+    const int nc = n_h * d_h, dq = d_h + d_r;
+    float w[8];
+    if (n0 < nc) {
+      const int h = n0 / d_h, i = n0 - h * d_h;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = qscale * v[k];
+      mla::store8(q + ((long long)m * n_h + h) * dq + i, w);
+      return;
+    }
+    const int j = n0 - nc, h = j / d_r, jj = j - h * d_r;
+    const int p = m % prefill_S;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float x0 = v[2 * k], x1 = v[2 * k + 1];
+      rope_rotate_pair(x0, x1, p, theta[(jj >> 1) + k]);
+      w[2 * k] = qscale * x0;
+      w[2 * k + 1] = qscale * x1;
+    }
+    mla::store8(q + ((long long)m * n_h + h) * dq + d_h + jj, w);
   }
 };
 

@@ -13,6 +13,7 @@
 
 #include <cudaTypedefs.h>
 
+#include "attn_mha.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -32,6 +33,7 @@ struct mla_weights {
   void* dq;            // [d_cq][d_model] or null
   void* uqr;           // [n_h*(d_h + d_r)][d_in]
   void* ukt;           // [n_h][d_c][d_h]
+  void* uk;            // [n_h*d_h][d_c] (as given: the materialised prefill expands K_C with it)
   void* uv;            // [n_h*d_v][d_c]
   double theta[32];    // RoPE frequencies, theta_i = base^(-2i/d_r)
 };
@@ -129,7 +131,7 @@ size_t esize(const mla_dims& d) { return d.dtype == MLA_BF16 ? 2 : 4; }
 int d_in(const mla_dims& d) { return d.d_cq > 0 ? d.d_cq : d.d_model; }
 
 struct WeightLayout {
-  size_t dkr, dq, uqr, ukt, uv, total;
+  size_t dkr, dq, uqr, ukt, uk, uv, total;
 };
 WeightLayout weight_layout(const mla_dims& d) {
   const size_t e = esize(d);
@@ -139,6 +141,7 @@ WeightLayout weight_layout(const mla_dims& d) {
   L.dq = o;  o = align_up(o + e * (size_t)d.d_cq * d.d_model, 256);
   L.uqr = o; o = align_up(o + e * (size_t)d.n_h * (d.d_h + d.d_r) * d_in(d), 256);
   L.ukt = o; o = align_up(o + e * (size_t)d.n_h * d.d_c * d.d_h, 256);
+  L.uk = o;  o = align_up(o + e * (size_t)d.n_h * d.d_h * d.d_c, 256);
   L.uv = o;  o = align_up(o + e * (size_t)d.n_h * d.d_v * d.d_c, 256);
   L.total = o;
   return L;
@@ -173,7 +176,7 @@ Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false) {
     P.rb_first = o;   o = align_up(o + sizeof(int) * (size_t)(R + 1), 256);
     P.split_rbs = o;  o = align_up(o + sizeof(int) * (size_t)(2 * W + 1), 256);
     P.part_o = o;     o = align_up(o + sizeof(float) * slots * d.n_h * d.d_c, 256);
-    P.part_ml = o;    o = align_up(o + sizeof(float) * slots * d.n_h * 2, 256);
+    P.part_ml = o;    o = align_up(o + sizeof(float) * slots * 2 * d.n_h * 2, 256);
     P.obar = o;       o = align_up(o + e * (size_t)R * d.n_h * d.d_c, 256);
   }
   P.total = o;
@@ -507,6 +510,120 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   return MLA_OK;
 }
 
+// ------------------------------------------------ materialised causal prefill
+// Workspace: the split-K scratch of the projections, then the token-ordered
+// cache rows, c_Q, the queries [T][n_h][d_h + d_r], K_C [T][n_h][d_h] and
+// V [T][n_h][d_v].
+struct MatPlan {
+  Plan base;   // hdr, counters, partial
+  size_t dense, cq, q, kc, v, total;
+};
+MatPlan make_mat_plan(const mla_dims& d, int T) {
+  MatPlan M{};
+  M.base = make_plan(d, T, false);
+  size_t o = M.base.total;
+  M.dense = o; o = align_up(o + 2 * (size_t)T * (d.d_c + d.d_r), 256);
+  M.cq = o;    o = align_up(o + 2 * (size_t)T * d.d_cq, 256);
+  M.q = o;     o = align_up(o + 2 * (size_t)T * d.n_h * (d.d_h + d.d_r), 256);
+  M.kc = o;    o = align_up(o + 2 * (size_t)T * d.n_h * d.d_h, 256);
+  M.v = o;     o = align_up(o + 2 * (size_t)T * d.n_h * d.d_v, 256);
+  M.total = o;
+  return M;
+}
+
+// Dimensions the materialised kernel takes: bf16, a 64-wide RoPE key, and
+// head widths that are whole 64-column chunks of at most 128.
+bool mat_supported(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.d_r == attn_mha::DR && (d.d_h == 64 || d.d_h == 128) &&
+         (d.d_v == 64 || d.d_v == 128);
+}
+
+mla_status prefill_mat_impl(const mla_weights* w, const void* h, const int32_t* page_table, int max_pages,
+                            int num_pages, void* cache, float* out, int B, int S, void* ws, const MatPlan& M,
+                            cudaStream_t st) {
+  using T = __nv_bfloat16;
+  const mla_dims& d = w->d;
+  const int T_ = B * S, d_cr = d.d_c + d.d_r, din = d_in(d), dq = d.d_h + d.d_r;
+  const Plan& P = M.base;
+  cudaError_t e;
+  // (1) append every token, keeping a token-ordered copy of the rows.
+  {
+    EpiAppend<T> epi{};
+    epi.cache = static_cast<T*>(cache);
+    epi.prefill_S = S;
+    epi.page_table = page_table;
+    for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
+    epi.max_pages = max_pages;
+    epi.num_pages = num_pages;
+    epi.page_size = d.page_size;
+    epi.d_c = d.d_c;
+    epi.d_cr = d_cr;
+    epi.n_seq = B;
+    epi.err = at<int>(ws, P.hdr);
+    epi.dense = at<T>(ws, M.dense);
+    if ((e = gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, d_cr, d.d_model, 1, epi, ws, P, st)))
+      return cuda_status(e);
+  }
+  // (2) query latent, (3) [q_C | RoPE(q_R)] per head, scaled by s * log2 e.
+  const void* src = h;
+  if (d.d_cq > 0) {
+    EpiStore<T> epi{at<T>(ws, M.cq), d.d_cq, 0, 1.f};
+    if ((e = gemm<T>(h, d.d_model, 0, w->dq, d.d_model, 0, T_, d.d_cq, d.d_model, 1, epi, ws, P, st)))
+      return cuda_status(e);
+    src = at<T>(ws, M.cq);
+  }
+  {
+    EpiQProjM<T> epi{};
+    epi.q = at<T>(ws, M.q);
+    for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
+    epi.n_h = d.n_h; epi.d_h = d.d_h; epi.d_r = d.d_r; epi.prefill_S = S;
+    epi.qscale = (float)((double)w->scale * kLog2e);
+    if ((e = gemm<T>(src, din, 0, w->uqr, din, 0, T_, d.n_h * (d.d_h + d.d_r), din, 1, epi, ws, P, st)))
+      return cuda_status(e);
+  }
+  // (4) expansion: K_C = W_UK c and V = W_UV c for every token and head.
+  {
+    EpiStore<T> ek{at<T>(ws, M.kc), (long long)d.n_h * d.d_h, 0, 1.f};
+    if ((e = gemm<T>(at<T>(ws, M.dense), d_cr, 0, w->uk, d.d_c, 0, T_, d.n_h * d.d_h, d.d_c, 1, ek, ws, P, st)))
+      return cuda_status(e);
+    EpiStore<T> ev{at<T>(ws, M.v), (long long)d.n_h * d.d_v, 0, 1.f};
+    if ((e = gemm<T>(at<T>(ws, M.dense), d_cr, 0, w->uv, d.d_c, 0, T_, d.n_h * d.d_v, d.d_c, 1, ev, ws, P, st)))
+      return cuda_status(e);
+  }
+  // (5) causal multi-head attention on the expanded keys and values.
+  CUtensorMap mq, mk, mv, mr;
+  if (!encode_bf16_3d(&mq, at<T>(ws, M.q), dq, d.n_h, T_, dq, (long long)d.n_h * dq, 64, 1, attn_mha::BQ) ||
+      !encode_bf16_3d(&mk, at<T>(ws, M.kc), d.d_h, d.n_h, T_, d.d_h, (long long)d.n_h * d.d_h, 64, 1,
+                      attn_mha::BKV) ||
+      !encode_bf16_3d(&mv, at<T>(ws, M.v), d.d_v, d.n_h, T_, d.d_v, (long long)d.n_h * d.d_v, 64, 1,
+                      attn_mha::BKV) ||
+      !encode_cache_map(&mr, cache, d_cr, (long long)num_pages * d.page_size, 64))
+    return MLA_ERR_CUDA;
+  attn_mha::Params pp{B, S, d.n_h, d.d_h, d.d_v, d.d_c, dq / 64, d.d_v / 64, page_table, max_pages, num_pages,
+                      out, at<int>(ws, P.hdr)};
+  if ((e = set_smem_once(attn_mha::attn_mha_kernel, attn_mha::SMEM_BYTES))) return cuda_status(e);
+  ++g_launches;
+  prof_mark(st, true);
+  attn_mha::attn_mha_kernel<<<dim3(ceil_div(S, attn_mha::BQ), d.n_h, B), attn_mha::THREADS, attn_mha::SMEM_BYTES,
+                              st>>>(mq, mk, mv, mr, pp);
+  prof_mark(st, false);
+  return cuda_status(cudaGetLastError());
+}
+
+// One warp waits on an mbarrier nobody arrives at; the bounded wait gives up
+// after limit_ns, records kErrTimeout in *err and the kernel returns.
+__global__ void wait_timeout_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::mbar_fence_init();
+  }
+  __syncwarp();
+  sm100::mbar_wait_warp(&bar, 0, &abort_flag, err, limit_ns);
+}
+
 mla_status begin_call(void* ws, cudaStream_t st, const Plan& P) {
   g_launches = 0;
   return cuda_status(cudaMemsetAsync(ws, 0, P.partial, st));  // header + split-K counters
@@ -603,6 +720,9 @@ mla_status mla_absorb_weights(const mla_dims* dims, const void* W_DKV, const voi
   if ((err = cudaMemcpyAsync(base + L.uv, W_UV, e * (size_t)d.n_h * d.d_v * d.d_c, cudaMemcpyDeviceToDevice,
                              stream)))
     return cuda_status(err);
+  if ((err = cudaMemcpyAsync(base + L.uk, W_UK, e * (size_t)d.n_h * d.d_h * d.d_c, cudaMemcpyDeviceToDevice,
+                             stream)))
+    return cuda_status(err);
   // Per-head transpose of W_UK: [n_h][d_h][d_c] -> [n_h][d_c][d_h].
   {
     dim3 grid(ceil_div(d.d_c, 32), ceil_div(d.d_h, 32), d.n_h);
@@ -624,6 +744,7 @@ mla_status mla_absorb_weights(const mla_dims* dims, const void* W_DKV, const voi
   w->dq = d.d_cq > 0 ? base + L.dq : nullptr;
   w->uqr = base + L.uqr;
   w->ukt = base + L.ukt;
+  w->uk = base + L.uk;
   w->uv = base + L.uv;
   for (int i = 0; i < d.d_r / 2; ++i) w->theta[i] = pow((double)d.rope_base, -2.0 * i / d.d_r);
   *out = w;
@@ -773,6 +894,27 @@ mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_
                             workspace, P, stream);
 }
 
+size_t mla_prefill_materialised_workspace_bytes(const mla_dims* dims, int B, int S) {
+  if (check_dims(dims) != MLA_OK || !mat_supported(*dims) || B <= 0 || S <= 0) return 0;
+  return make_mat_plan(*dims, B * S).total;
+}
+
+mla_status mla_prefill_materialised(const mla_weights* w, const void* h, const int32_t* page_table, int max_pages,
+                                    int num_pages, void* cache, float* out, int B, int S, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || B <= 0 || S <= 0 || max_pages <= 0 || num_pages <= 0) return MLA_ERR_INVALID_ARG;
+  if (!mat_supported(w->d)) return MLA_ERR_UNSUPPORTED;
+  if (!h || !page_table || !cache || !out || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)max_pages * w->d.page_size < S || (long long)B * S > INT_MAX / 2) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h, 16) || !aligned(cache, 16) || !aligned(out, 16))
+    return MLA_ERR_INVALID_ARG;
+  const MatPlan M = make_mat_plan(w->d, B * S);
+  if (workspace_bytes < M.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, M.base);
+  if (s != MLA_OK) return s;
+  return prefill_mat_impl(w, h, page_table, max_pages, num_pages, cache, out, B, S, workspace, M, stream);
+}
+
 mla_status mla_get_error(const void* workspace, cudaStream_t stream) {
   if (!workspace) return MLA_ERR_INVALID_ARG;
   int word = 0;
@@ -783,6 +925,16 @@ mla_status mla_get_error(const void* workspace, cudaStream_t stream) {
   if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
   if (word & kErrBounds) return MLA_ERR_DEVICE_BOUNDS;
   return MLA_OK;
+}
+
+mla_status mla_selftest_wait_timeout(void* workspace, int limit_us, cudaStream_t stream) {
+  if (!workspace || !aligned(workspace, 256) || limit_us < 1 || limit_us > 1000000) return MLA_ERR_INVALID_ARG;
+  g_launches = 0;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  ++g_launches;
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<int*>(workspace), 1000ull * (unsigned long long)limit_us);
+  return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"
@@ -810,7 +962,7 @@ namespace {
 
 constexpr int kNoAllocMaxT = 256;                 // tokens per call
 constexpr int kNoAllocTileSplits = 128;           // split-K tiles x splits
-constexpr size_t kNoAllocHdr = 256;               // unused error word slot
+constexpr size_t kNoAllocHdr = 256;               // error word: takes device errors when device_error is NULL (then discarded)
 constexpr size_t kNoAllocCounters = sizeof(int) * kCounterCap;
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocHdr + kNoAllocCounters + sizeof(float) * (size_t)kNoAllocTileSplits * 64 * 64;

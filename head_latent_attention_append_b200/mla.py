@@ -26,6 +26,7 @@ EXPORTED = [
     "mla_prefill_workspace_bytes", "mla_prefill", "mla_get_error", "mla_status_string",
     "mla_last_launch_count", "mla_profile_begin", "mla_profile_end", "mla_append_latent_noalloc",
     "mla_decode_cp_workspace_bytes", "mla_decode_cp_partial", "mla_decode_cp_combine",
+    "mla_selftest_wait_timeout", "mla_prefill_materialised_workspace_bytes", "mla_prefill_materialised",
 ]
 APPEND_NOALLOC_MAX_T = 256
 
@@ -74,6 +75,9 @@ def _load():
         "mla_decode_cp_workspace_bytes": (Z, [D, I, I]),
         "mla_decode_cp_partial": (S, [P, P, P, P, P, P, I, I, P, P, P, I, I, I, P, Z, P]),
         "mla_decode_cp_combine": (S, [P, I, P, P, P, I, I, P, Z, P]),
+        "mla_selftest_wait_timeout": (S, [P, I, P]),
+        "mla_prefill_materialised_workspace_bytes": (Z, [D, I, I]),
+        "mla_prefill_materialised": (S, [P, P, P, I, I, P, P, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -196,6 +200,18 @@ def prefill(w: Weights, h, page_table, num_pages: int, cache, out, workspace, st
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def prefill_materialised_workspace_bytes(dims: Dims, B: int, S: int) -> int:
+    return lib.mla_prefill_materialised_workspace_bytes(ctypes.byref(dims), B, S)
+
+
+def prefill_materialised(w: Weights, h, page_table, num_pages: int, cache, out, workspace, stream=None):
+    """Causal prefill through expanded per-head keys and values (include/mla.h)."""
+    B, S = h.shape[0], h.shape[1]
+    _check("mla_prefill_materialised", lib.mla_prefill_materialised(
+        w.handle, _ptr(h), _ptr(page_table), page_table.shape[1], num_pages, _ptr(cache), _ptr(out), B, S,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def decode_cp_workspace_bytes(dims: Dims, B: int, n_q: int) -> int:
     return lib.mla_decode_cp_workspace_bytes(ctypes.byref(dims), B, n_q)
 
@@ -216,6 +232,11 @@ def decode_cp_combine(w: Weights, obar_parts, lse_parts, out, workspace, stream=
     _check("mla_decode_cp_combine", lib.mla_decode_cp_combine(
         w.handle, n_ranks, _ptr(obar_parts), _ptr(lse_parts), _ptr(out), B, n_q, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def selftest_wait_timeout(workspace, limit_us: int, stream=None):
+    """Test hook: a bounded wait that nothing satisfies (include/mla.h)."""
+    _check("mla_selftest_wait_timeout", lib.mla_selftest_wait_timeout(_ptr(workspace), limit_us, _stream(stream)))
 
 
 def get_error(workspace, stream=None) -> int:

@@ -48,10 +48,19 @@ class Workload:
     ragged: bool = False
     max_cached: int = 0     # ragged: lengths drawn from U{1..max_cached}
     rope_base: float = 10000.0
+    materialised: bool = False  # prefill through expanded per-head keys and values
 
     @property
     def d_cr(self) -> int:
         return self.d_c + self.d_r
+
+    def flops_per_pair(self) -> int:
+        """Algorithmic flops per causal (query, key) pair, all heads: the
+        absorbed form scores over d_c + d_r columns and sums d_c latent
+        columns; the materialised form scores over d_h + d_r and sums d_v."""
+        if self.materialised:
+            return self.n_h * (2 * (self.d_h + self.d_r) + 2 * self.d_v)
+        return self.n_h * (2 * self.d_cr + 2 * self.d_c)
 
 
 WORKLOADS = {
@@ -65,6 +74,9 @@ WORKLOADS = {
         # Multi-token (speculative-style) decode: 4 new tokens per sequence over ragged histories.
         Workload("dsv2_spec4_decode", 6, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "decode", 64, 4, 0,
                  ragged=True, max_cached=32768),
+        # The causal prefill of config 4 (same seeds, same inputs) in the materialised form.
+        Workload("dsv2_bf16_prefill_mat", 4, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "prefill", 4, 4096, 0,
+                 materialised=True),
     ]
 }
 

@@ -75,21 +75,26 @@ class Setup:
         keys = wl.B * wl.n_q if wl.mode == "prefill" else int(self.kv_len_host.sum())
         return keys * wl.d_cr * esz
 
-    def attention_flops(self) -> int:
+    def attention_pairs(self) -> int:
+        """Causal (query, key) pairs of one step."""
         wl = self.wl
         if wl.mode == "prefill":
-            pairs = wl.B * wl.n_q * (wl.n_q + 1) // 2
-        else:
-            pairs = int(sum(int(L) - wl.n_q + 1 + q for L in self.kv_len_host for q in range(wl.n_q)))
-        return pairs * wl.n_h * (2 * wl.d_cr + 2 * wl.d_c)
+            return wl.B * wl.n_q * (wl.n_q + 1) // 2
+        return int(sum(int(L) - wl.n_q + 1 + q for L in self.kv_len_host for q in range(wl.n_q)))
+
+    def attention_flops(self) -> int:
+        """The step's algorithmic attention flops in its own form (absorbed or
+        materialised)."""
+        return Setup.attention_pairs(self) * self.wl.flops_per_pair()
 
 
 def setup(name: str, device="cuda", checked_count: int = 4, check_all: Optional[bool] = None,
-          seed: int = synth.BASE_SEED, build_history: bool = True) -> Setup:
+          seed: int = synth.BASE_SEED, build_history: bool = True, softmax_scale: float = 0.0) -> Setup:
+    """``softmax_scale`` 0 selects the library default 1/sqrt(d_h + d_r)."""
     wl = synth.WORKLOADS[name]
     dev = torch.device(device)
     dt = TORCH_DTYPE[wl.dtype]
-    dims = dims_of(wl)
+    dims = dims_of(wl, softmax_scale)
     hw = synth.make_weights(wl, seed)
     W = upload_weights(wl, hw, dev)
     weights = mla.Weights(dims, W)
@@ -116,7 +121,9 @@ def setup(name: str, device="cuda", checked_count: int = 4, check_all: Optional[
                 synth.device_fill_normal_(h_new[b], seed * 1000 + b)
         cache.zero_()
         out = torch.empty((wl.B, S, wl.n_h, wl.d_v), dtype=torch.float32, device=dev)
-        ws = torch.empty(mla.prefill_workspace_bytes(dims, wl.B, S), dtype=torch.uint8, device=dev)
+        nws = (mla.prefill_materialised_workspace_bytes(dims, wl.B, S) if wl.materialised
+               else mla.prefill_workspace_bytes(dims, wl.B, S))
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev)
         return Setup(wl, dims, hw, weights, kv, layout, kv_len, page_table, cache, h_new, None, None, out, None,
                      ws, checked, host_hidden)
 
@@ -162,7 +169,8 @@ def step(s: Setup, stream=None) -> int:
     or append every token and attend causally (prefill).  Returns the number
     of kernels libmla launched."""
     if s.wl.mode == "prefill":
-        mla.prefill(s.weights, s.h_new, s.page_table, s.layout.num_pages, s.cache, s.out, s.ws, stream)
+        fn = mla.prefill_materialised if s.wl.materialised else mla.prefill
+        fn(s.weights, s.h_new, s.page_table, s.layout.num_pages, s.cache, s.out, s.ws, stream)
         return mla.last_launch_count()
     wl = s.wl
     mla.append_latent(s.weights, s.h_new.view(wl.B * wl.n_q, wl.d_model), s.seq_idx, s.pos, s.page_table,

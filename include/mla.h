@@ -234,6 +234,29 @@ mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Causal prefill in the materialised form ("Multi-Head Latent Attention"
+ * (talalahmed), "Compress first, expand later" and its closing flow diagram):
+ * the same result as mla_prefill, computed by expanding every token's latent
+ * into per-head keys K_C = W_UK,h c_t and values V = W_UV,h c_t and running
+ * causal multi-head attention on [K_C | k_R] (d_h + d_r columns) and V, so the
+ * output needs no W_UV after the sum.  It does 2 (d_h + d_r) + 2 d_v flops
+ * per (query, key) pair and head instead of 2 (d_c + d_r) + 2 d_c, at the cost
+ * of writing and reading the expanded K_C and V.  Absorbed and materialised
+ * results agree to rounding, not bit for bit (the order of the products
+ * differs; "ropeabsorb", "Absorption is exact").
+ * Arguments, layouts and the cache append are those of mla_prefill.  Supports
+ * bf16 with d_r = 64, d_h in {64, 128} and d_v in {64, 128}; other dimensions
+ * return MLA_ERR_UNSUPPORTED (the size query returns 0).
+ * Workspace: mla_prefill_materialised_workspace_bytes(dims, B, S) (it holds the
+ * expanded K_C and V: 2 * B * S * n_h * (d_h + d_v) bytes of it).
+ * ------------------------------------------------------------------------- */
+size_t mla_prefill_materialised_workspace_bytes(const mla_dims* dims, int B, int S);
+mla_status mla_prefill_materialised(const mla_weights* w, const void* h, const int32_t* page_table,
+                                    int max_pages, int num_pages, void* cache, float* out, int B,
+                                    int S, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status.
  * ------------------------------------------------------------------------- */
 /* Waits for `stream`, then returns the error recorded on the device by the
@@ -242,6 +265,18 @@ mla_status mla_prefill(const mla_weights* w, const void* h, const int32_t* page_
  * of range), or MLA_ERR_UNSUPPORTED (the device placed the attention
  * kernel's shared memory off the 1024-byte alignment it relies on). */
 mla_status mla_get_error(const void* workspace, cudaStream_t stream);
+
+/* Test hook for the failure path (the pages have no counterpart).  Launches
+ * one warp that waits, bounded by limit_us microseconds, on an mbarrier that
+ * nothing ever arrives at.  When the bound runs out the wait records
+ * MLA_ERR_TIMEOUT in the error word of `workspace` exactly as the library's
+ * pipelined kernels do on a stalled pipeline, and the kernel returns; no copy
+ * or MMA is in flight, so the context stays usable.  mla_get_error(workspace)
+ * then reports MLA_ERR_TIMEOUT.  workspace: device memory of at least 256
+ * bytes, 256-byte aligned; its error word is zeroed first.  Errors:
+ * MLA_ERR_INVALID_ARG (null or misaligned workspace, limit_us outside
+ * [1, 1000000]), MLA_ERR_CUDA. */
+mla_status mla_selftest_wait_timeout(void* workspace, int limit_us, cudaStream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char* mla_status_string(mla_status s);

@@ -31,6 +31,12 @@ section):
 * Context-parallel decode (``window_partial``, ``merge_windows``,
   ``latent_output``).  The pages do not split a sequence over devices; these
   state the softmax-over-disjoint-key-sets identity a split relies on.
+* Per-head position keys (``rope_per_head``).  The 16-head example of
+  "Multi-Head Latent Attention" (talalahmed), section "A concrete size
+  comparison", caches one 32-dim RoPE key per head instead of one shared key:
+  ``k_R,h,t = RoPE_t(W_KR,h h_t)`` with ``W_KR`` then ``[n_h*d_r, D]`` (rows
+  ``h*d_r ..`` for head ``h``), and head ``h``'s position term is
+  ``q_R,h . k_R,h,t``.  Everything else is unchanged.
 * RoPE.  Pairs ``(2i, 2i+1)`` rotated by angle ``pos * theta_i`` with
   ``theta_i = base^(-2i/d_r)``; the pages print only the rotation family and its
   relative property ``R_m^T R_t = R_{t-m}`` ("ai-decoupled-rope-mla", decoupled
@@ -70,6 +76,7 @@ class Dims:
     d_model: int
     d_cq: int = 0           # 0: the query is projected straight from h
     rope_base: float = 10000.0
+    rope_per_head: bool = False  # one RoPE key per head (W_KR is [n_h*d_r, D]) instead of one shared
 
     @property
     def d_in(self) -> int:
@@ -147,11 +154,26 @@ def rope_apply(x: np.ndarray, pos: np.ndarray, freqs: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 def cache_entries(w: Weights, H: np.ndarray, pos: np.ndarray, freqs: np.ndarray):
     """The two cached quantities per token: the latent ``c_t = W_DKV h_t`` and
-    the shared, already rotated position key ``RoPE_t(W_KR h_t)``."""
+    the already rotated position key ``RoPE_t(W_KR h_t)``: one shared key
+    ``[T, d_r]`` when ``W_KR`` has ``d_r`` rows, else one per head
+    ``[T, n_h, d_r]`` (``W_KR`` with ``n_h*d_r`` rows, head ``h`` at rows
+    ``h*d_r ..``)."""
     H = np.asarray(H, dtype=np.float64)
     c = H @ w.W_DKV.T
-    k_r = rope_apply(H @ w.W_KR.T, pos, freqs)
-    return c, k_r
+    d_r = 2 * len(freqs)
+    k = H @ np.asarray(w.W_KR, np.float64).T
+    if k.shape[1] == d_r:
+        return c, rope_apply(k, pos, freqs)
+    k = k.reshape(H.shape[0], k.shape[1] // d_r, d_r)
+    return c, rope_apply(k, np.asarray(pos)[:, None], freqs)
+
+
+def _position_term(q_r, k_r):
+    """``q_R,h . k_R,t`` for every query, head and key: ``[Q, n_h, T]``; the key
+    is shared ``[T, d_r]`` or per head ``[T, n_h, d_r]``."""
+    if k_r.ndim == 2:
+        return np.matmul(q_r, k_r.T)
+    return np.einsum("qhr,thr->qht", q_r, k_r)
 
 
 def queries(w: Weights, dims: Dims, H: np.ndarray, pos: np.ndarray, freqs: np.ndarray):
@@ -192,7 +214,7 @@ def attend_materialised(dims: Dims, w: Weights, q_c, q_r, c, k_r, q_pos, k_pos,
     k_pos = np.asarray(k_pos)
     visible = k_pos[None, :] <= q_pos[:, None]                    # [Q, T]
     out = np.empty((q_c.shape[0], n_h, d_v))
-    pos_term = np.matmul(q_r, k_r.T)                              # [Q, n_h, T]
+    pos_term = _position_term(q_r, k_r)                           # [Q, n_h, T]
     for h0 in range(0, n_h, head_chunk):
         hs = slice(h0, min(n_h, h0 + head_chunk))
         k_c = np.matmul(c[None], W_UK[hs].transpose(0, 2, 1))     # [h, T, d_h]  (K_C = W_UK,h c_t)
@@ -214,7 +236,7 @@ def attend_absorbed(dims: Dims, w: Weights, q_c, q_r, c, k_r, q_pos, k_pos,
     W_UK = w.W_UK.reshape(n_h, d_h, d_c)
     W_UV = w.W_UV.reshape(n_h, d_v, d_c)
     q_abs = np.einsum("qhd,hdc->qhc", q_c, W_UK)
-    a = (np.einsum("qhc,tc->qht", q_abs, c) + np.einsum("qhr,tr->qht", q_r, k_r)) * scale
+    a = (np.einsum("qhc,tc->qht", q_abs, c) + _position_term(q_r, k_r)) * scale
     visible = np.asarray(k_pos)[None, :] <= np.asarray(q_pos)[:, None]
     a = np.where(visible[:, None, :], a, -np.inf)
     alpha = _softmax(a)
@@ -275,6 +297,7 @@ def window_partial(dims: Dims, w: Weights, H: np.ndarray, n_q: int, start: int, 
     latent sum over those keys (scores against the latent with the absorbed
     query ``q~ = W_UK,h^T q_C``) and ``log2 sum_t exp(a_t)``.  A query with no
     such key gets ``o_bar = 0`` and ``lse2 = -inf``."""
+    assert not dims.rope_per_head, "window partials are stated for the shared position key"
     w = as_f64(w)
     H = np.asarray(H, dtype=np.float64)
     T = H.shape[0]
@@ -348,7 +371,12 @@ def brute_force_sequence(dims: Dims, w: Weights, H, query_rows, scale=None):
         return y
 
     c = [matvec(Wl["W_DKV"], Hl[t]) for t in range(T)]
-    kr = [rot(matvec(Wl["W_KR"], Hl[t]), t) for t in range(T)]
+    kr_all = [matvec(Wl["W_KR"], Hl[t]) for t in range(T)]
+
+    def key(t, h):
+        """Head h's rotated position key of token t (shared or its own)."""
+        base = h * d_r if dims.rope_per_head else 0
+        return rot(kr_all[t][base:base + d_r], t)
     out = []
     for m in query_rows:
         src = matvec(Wl["W_DQ"], Hl[m]) if dims.d_cq > 0 else Hl[m]
@@ -362,7 +390,8 @@ def brute_force_sequence(dims: Dims, w: Weights, H, query_rows, scale=None):
             for t in range(m + 1):
                 kc = [sum(Wl["W_UK"][h * d_h + i][j] * c[t][j] for j in range(d_c)) for i in range(d_h)]
                 v = [sum(Wl["W_UV"][h * d_v + i][j] * c[t][j] for j in range(d_c)) for i in range(d_v)]
-                s = sum(qc[i] * kc[i] for i in range(d_h)) + sum(qr[i] * kr[t][i] for i in range(d_r))
+                kr = key(t, h)
+                s = sum(qc[i] * kc[i] for i in range(d_h)) + sum(qr[i] * kr[i] for i in range(d_r))
                 scores.append(s * scale)
                 vals.append(v)
             mx = max(scores)

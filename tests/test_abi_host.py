@@ -58,6 +58,12 @@ def test_size_queries(mla):
     assert mla.decode_cp_workspace_bytes(d, 1024, 1) > mla.decode_workspace_bytes(d, 1024, 1, 8193)
     assert mla.decode_cp_workspace_bytes(dims3(mla, dtype=mla.F32), 4, 1) == 0
     assert mla.decode_cp_workspace_bytes(d, 0, 1) == 0
+    # Materialised prefill: bf16, d_r = 64, d_h and d_v in {64, 128}; it holds the expanded K_C and V.
+    assert mla.prefill_materialised_workspace_bytes(d, 4, 4096) >= 2 * 4 * 4096 * 128 * (128 + 128)
+    assert mla.prefill_materialised_workspace_bytes(dims3(mla, d_r=32), 4, 4096) == 0
+    assert mla.prefill_materialised_workspace_bytes(dims3(mla, d_h=96), 4, 4096) == 0
+    assert mla.prefill_materialised_workspace_bytes(dims3(mla, dtype=mla.F32), 4, 4096) == 0
+    assert mla.prefill_materialised_workspace_bytes(d, 0, 4096) == 0
 
 
 def test_status_strings(mla):
@@ -98,6 +104,11 @@ def test_bad_arguments_are_rejected_before_launch(mla):
     assert lib.mla_decode_cp_combine(None, 2, FAKE, FAKE, FAKE, 1, 1, FAKE, 1 << 30, None) == -1
     assert lib.mla_get_error(None, None) == -1
     assert lib.mla_weights_dims(None, ctypes.byref(d)) == -1
+    # The timeout self-test hook: null or misaligned workspace, limit out of range.
+    assert lib.mla_selftest_wait_timeout(None, 1000, None) == -1
+    assert lib.mla_selftest_wait_timeout(FAKE + 8, 1000, None) == -1
+    assert lib.mla_selftest_wait_timeout(FAKE, 0, None) == -1
+    assert lib.mla_selftest_wait_timeout(FAKE, 1000001, None) == -1
 
 
 def test_handle_arguments_checked_before_launch(mla):

@@ -56,3 +56,15 @@ def test_headline_figures_of_the_decode_and_prefill_workloads():
     wp = synth.WORKLOADS["dsv2_bf16_prefill"]
     sp = _setup(wp, np.zeros(wp.B, np.int32))
     assert workload.Setup.attention_flops(sp) == 33_562_624 * 278_528     # 9.348 TFLOP over the causal pairs
+
+
+def test_materialised_prefill_counts_its_own_flops():
+    """The materialised twin of the prefill workload scores over d_h + d_r
+    columns and sums d_v: 640 flops per pair and head instead of 2176."""
+    wm = synth.WORKLOADS["dsv2_bf16_prefill_mat"]
+    wp = synth.WORKLOADS["dsv2_bf16_prefill"]
+    assert wm.materialised and not wp.materialised
+    assert (wm.B, wm.n_q, wm.wid) == (wp.B, wp.n_q, wp.wid)         # the same inputs
+    sm = _setup(wm, np.zeros(wm.B, np.int32))
+    assert wm.flops_per_pair() == 128 * (2 * (128 + 64) + 2 * 128) == 81_920
+    assert workload.Setup.attention_flops(sm) == 33_562_624 * 81_920      # 2.749 TFLOP

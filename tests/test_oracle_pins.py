@@ -257,3 +257,90 @@ def test_cache_sizes_printed_on_the_pages():
             assert round(mha / mla) == pytest.approx(e["ratio"], abs=1.0)
         if "reduction" in e:
             assert 1 - mla / mha == pytest.approx(e["reduction"], abs=0.01)
+
+
+# --------------------------------------------- per-head position keys -----
+# The 16-head example of "Multi-Head Latent Attention" (talalahmed), "A
+# concrete size comparison", caches one RoPE key per head.
+import dataclasses  # noqa: E402
+
+TINY_PH = dataclasses.replace(TINY, rope_per_head=True)
+SMALL_PH = dataclasses.replace(SMALL, rope_per_head=True)
+
+
+def per_head_weights(rng, dims):
+    w = rand_weights(rng, dataclasses.replace(dims, rope_per_head=False))
+    w.W_KR = rng.standard_normal((dims.n_h * dims.d_r, dims.d_model)) / math.sqrt(dims.d_model)
+    return w
+
+
+def test_per_head_keys_reduce_to_the_shared_key_when_every_block_is_the_same():
+    rng = np.random.default_rng(20)
+    w = rand_weights(rng, SMALL)
+    H = rng.standard_normal((25, SMALL.d_model))
+    rows = [0, 12, 24]
+    w_ph = dataclasses.replace(w, W_KR=np.tile(w.W_KR, (SMALL.n_h, 1)))
+    shared = O.mla_sequence(SMALL, w, H, rows)
+    per_head = O.mla_sequence(SMALL_PH, w_ph, H, rows)
+    np.testing.assert_allclose(per_head, shared, rtol=0, atol=1e-13 * np.abs(shared).max())
+
+
+def test_per_head_keys_brute_force_tiny():
+    rng = np.random.default_rng(21)
+    w = per_head_weights(rng, TINY_PH)
+    H = rng.standard_normal((6, TINY_PH.d_model))
+    rows = [0, 2, 5]
+    ref = O.brute_force_sequence(TINY_PH, w, H, rows)
+    got = O.mla_sequence(TINY_PH, w, H, rows)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-13 * np.abs(ref).max())
+
+
+def test_per_head_keys_absorbed_equals_materialised():
+    rng = np.random.default_rng(22)
+    w = per_head_weights(rng, SMALL_PH)
+    H = rng.standard_normal((30, SMALL_PH.d_model))
+    a = O.mla_sequence(SMALL_PH, w, H, [3, 29], absorbed=True)
+    m = O.mla_sequence(SMALL_PH, w, H, [3, 29])
+    assert np.abs(a - m).max() / np.abs(m).max() <= 1e-12
+    assert not np.array_equal(a, m)
+
+
+def test_per_head_keys_keep_the_relative_property():
+    rng = np.random.default_rng(23)
+    w = per_head_weights(rng, SMALL_PH)
+    H = rng.standard_normal((18, SMALL_PH.d_model))
+    base = O.mla_sequence(SMALL_PH, w, H, [17])
+    shifted = O.mla_sequence(SMALL_PH, w, H, [17], positions=np.arange(18) + 4321)
+    assert np.abs(shifted - base).max() / np.abs(base).max() <= 1e-10
+
+
+def test_per_head_keys_use_each_heads_own_block():
+    """Distinct blocks change every head's scores: the result differs from the
+    shared-key result built from head 0's block, and head h's output depends
+    only on block h (replacing block 1 leaves head 0 unchanged)."""
+    rng = np.random.default_rng(24)
+    w = per_head_weights(rng, SMALL_PH)
+    H = rng.standard_normal((22, SMALL_PH.d_model))
+    got = O.mla_sequence(SMALL_PH, w, H, [21])
+    w0 = dataclasses.replace(w, W_KR=w.W_KR[:SMALL.d_r])
+    assert np.abs(got - O.mla_sequence(SMALL, w0, H, [21])).max() / np.abs(got).max() > 1e-3
+    W2 = w.W_KR.copy()
+    W2[SMALL.d_r:2 * SMALL.d_r] = rng.standard_normal((SMALL.d_r, SMALL.d_model))
+    got2 = O.mla_sequence(SMALL_PH, dataclasses.replace(w, W_KR=W2), H, [21])
+    np.testing.assert_array_equal(got2[:, 0], got[:, 0])
+    assert not np.allclose(got2[:, 1], got[:, 1])
+
+
+def test_per_head_cache_row_matches_the_pages_16_head_example():
+    """cache_entries of the 16-head example stores d_c + n_h * d_r = 768
+    numbers per token: the per-head size the page prints."""
+    with open(os.path.join(GOLDEN, "cache_sizes.json")) as fh:
+        ent = [e for e in json.load(fh)["entries"] if not e["shared_rope_key"]][0]
+    dims = O.Dims(n_h=ent["n_h"], d_h=ent["d_h"], d_v=ent["d_v"], d_c=ent["d_c"], d_r=ent["d_r"], d_model=40,
+                  rope_per_head=True)
+    rng = np.random.default_rng(25)
+    w = per_head_weights(rng, dims)
+    c, k_r = O.cache_entries(O.as_f64(w), rng.standard_normal((3, 40)), np.arange(3),
+                             O.rope_frequencies(dims.d_r, dims.rope_base))
+    assert k_r.shape == (3, dims.n_h, dims.d_r)
+    assert c.shape[1] + k_r[0].size == ent["mla"] == 768
