@@ -271,7 +271,8 @@ def oracle_sample(name: str, k: int = 0):
     order = [med] + [int(i) for i in np.random.default_rng(wl.wid).permutation(len(kv)) if i != med]
     b = order[k % len(order)]
     hw = synth.make_weights(wl)
-    dims = O.Dims(wl.n_h, wl.d_h, wl.d_v, wl.d_c, wl.d_r, wl.d_model, wl.d_cq, wl.rope_base)
+    dims = O.Dims(wl.n_h, wl.d_h, wl.d_v, wl.d_c, wl.d_r, wl.d_model, wl.d_cq, wl.rope_base,
+                  rope_per_head=wl.rope_per_head)
     w = O.Weights(**hw.as_dict())
     if wl.mode == "prefill":
         L = nq = min(PREFILL_SAMPLE_TOKENS, int(kv[b]))
@@ -537,6 +538,7 @@ def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
     d2h = s.out.numel() * s.out.element_size()
     res = {
         "workload": wl.name, "value": value, "unit": unit, "ms_per_step": ms_step,
+        "cache_bytes_per_token": wl.d_cr * (2 if wl.dtype == "bf16" else 4),
         "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "config": {"workload": wl.name, "B": wl.B, "n_q": wl.n_q, "kv_len": int(s.kv_len_host.max()),
                    "n_h": wl.n_h, "d_c": wl.d_c, "d_r": wl.d_r, "d_model": wl.d_model, "d_cq": wl.d_cq,
@@ -569,7 +571,8 @@ def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
 # causal prefill (the prefill TFLOP/s half of the metric) and the ragged
 # paged decode.
 EXTRA = {"prefill": "dsv2_bf16_prefill", "ragged": "dsv2_ragged_decode",
-         "prefill_materialised": "dsv2_bf16_prefill_mat"}
+         "prefill_materialised": "dsv2_bf16_prefill_mat", "page": "page_bf16_decode",
+         "page_per_head_rope": "page_bf16_decode_rph"}
 
 
 def run_ours(args):

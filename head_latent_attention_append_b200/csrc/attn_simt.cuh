@@ -2,7 +2,10 @@
 //
 // This is the fp32 path (the fp32 workload's 1e-4 bound rules out single-pass
 // TF32 on the tensor cores).  Per query token and head it computes
-//   a_t   = Q_abs[h] . cache[t]          over the d_c + d_r columns
+//   a_t   = Q_abs[h] . cache[t]          over the d_c latent columns and
+//           the d_r columns of the RoPE key (the shared one, or head h's own
+//           in the per-head layout of "Multi-Head Latent Attention",
+//           "A concrete size comparison")
 //           (Q_abs = [s*log2(e)*W_UK,h^T q_C,h | s*log2(e)*RoPE_m(q_R,h)], so
 //           a_t is the pages' score in log2 units)
 //   alpha = softmax over the visible keys (exp2, online, running max)
@@ -18,12 +21,14 @@
 namespace mla {
 
 struct AttnArgs {
-  const void* qabs;          // [R][qrows][d_cr]
+  const void* qabs;          // [R][qrows][q_row]
   int qrows;
-  const void* cache;         // [num_pages][page_size][d_cr]
+  const void* cache;         // [num_pages][page_size][d_cr]: a row is [c | k_R] (one shared key or n_h keys)
   const int32_t* page_table; // [n_seq][max_pages]
   int max_pages, num_pages, page_size;
   int n_h, d_c, d_r, d_cr;
+  int q_row;                 // Q_abs row: d_c + d_r ([q~ | q_R])
+  int rope_per_head;         // 0: one shared RoPE key per row; 1: head h's key at d_c + h*d_r
   const int32_t* kv_len;
   int uniform_kv_len, n_q, max_kv_len;
   Sched sched;
@@ -47,7 +52,7 @@ constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
 template <typename T>
 __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) {
   extern __shared__ float smem[];
-  const int pitch = a.d_cr + 1;
+  const int pitch = a.d_cr + 1;        // cache rows; a Q row uses the first q_row of its pitch
   float* Qs = smem;                    // [HG][pitch]
   float* Cs = Qs + HG * pitch;         // [KC][pitch]
   float* Ps = Cs + KC * pitch;         // [HG][KC]
@@ -66,9 +71,9 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
     const int rb = g.rb, seq = rb / a.n_q;
     const int nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
     __syncthreads();
-    for (int i = tid; i < HG * a.d_cr; i += THREADS) {
-      int h = i / a.d_cr, j = i % a.d_cr;
-      Qs[h * pitch + j] = (h0 + h < a.n_h) ? to_f32(qabs[((long long)rb * a.qrows + h0 + h) * a.d_cr + j]) : 0.f;
+    for (int i = tid; i < HG * a.q_row; i += THREADS) {
+      int h = i / a.q_row, j = i % a.q_row;
+      Qs[h * pitch + j] = (h0 + h < a.n_h) ? to_f32(qabs[((long long)rb * a.qrows + h0 + h) * a.q_row + j]) : 0.f;
     }
     if (tid < HG) {
       st[tid * 3 + 0] = -INFINITY;
@@ -101,8 +106,10 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
         int h = i / KC, k = i % KC;
         const float* q = Qs + h * pitch;
         const float* c = Cs + k * pitch;
+        const float* kr = c + a.d_c + (a.rope_per_head ? (h0 + h) * a.d_r : 0);
         float acc = 0.f;
-        for (int j = 0; j < a.d_cr; ++j) acc = fmaf(q[j], c[j], acc);
+        for (int j = 0; j < a.d_c; ++j) acc = fmaf(q[j], c[j], acc);
+        for (int j = 0; j < a.d_r; ++j) acc = fmaf(q[a.d_c + j], kr[j], acc);
         Ps[h * KC + k] = (k0 + k < k_end) ? acc : -INFINITY;
       }
       __syncthreads();

@@ -23,13 +23,9 @@
 // steps and, for d_r = 32 or 64, equal.  Each CTA streams only its own
 // columns of every page (no byte is read twice from HBM) and computes the
 // partial score over them into TMEM.  The partial goes to the peer as fp16
-// (saturated at +-65504, log2 units) through distributed shared memory, in
-// the 128-byte-swizzled K-major layout a tensor-core operand has, and each
-// CTA's tensor core adds the peer's partial to its own with one more MMA
-// against a 64 x 64 identity matrix: S = S_own + X_peer * I, exact in the
-// fp32 accumulator.  So the softmax threads read finished fp32 scores from
-// TMEM and do no conversion work.  Each CTA keeps its own exact partial, so
-// the two CTAs' scores differ by the rounding of one fp16 partial and each
+// (saturated at +-65504, log2 units) through distributed shared memory; each
+// CTA's softmax threads add the peer's partial to their own exact fp32 one.
+// So the two CTAs' scores differ by the rounding of one fp16 partial and each
 // runs its own softmax state (m, l) for its half of the latent columns: each
 // half is normalised by its own state, and split row blocks leave one
 // (m, l) per half.  fp16's 11-bit significand keeps this well below the
@@ -38,17 +34,18 @@
 //
 // TMEM columns: O [0, d_c/2), two score buffers S0 [256, 320) and
 // S1 [320, 384), the latent part of this CTA's Q slice from 384 (at most 128
-// columns).  A score buffer is free again as soon as the finishers have read
-// it; P (bf16) goes to a shared-memory tile that the SS P*V MMA reads.
+// columns).  A score buffer is free again as soon as the sender and the
+// finishers have read it (the peer's partial is not waited for first), so the
+// DSMEM latency of the exchange stays out of the score pipeline.
 //
 // Shared memory (1024-byte aligned pieces):
-//   three 16 KB exchange buffers, written by the peer's sender threads with
-//     asynchronous remote stores (st.async, 16 bytes each, straight from
-//     registers) that complete on this CTA's mbarrier; the MMA that consumes
-//     one returns it to the peer with a tcgen05.commit multicast onto the
-//     peer's credit barrier.  (A staged bulk copy goes through the TMA engine
-//     behind the page loads and landed ~1.6 us after issue; the remote
-//     stores skip that queue.);
+//   three 16 KB exchange buffers, filled by the peer with bulk copies (one
+//     4 KB copy per sender warp per page) that complete on this CTA's
+//     mbarrier; each goes back to the peer with a tcgen05.commit multicast
+//     onto the peer's credit barrier after the page's P*V, which is issued
+//     only once the finishers have read the buffer (a remote arrive from the
+//     finishers themselves is a cluster-scope release that stalls the warp);
+//   a 16 KB staging block for this CTA's outgoing partial;
 //   score ring, 2 slots: this CTA's columns of a page (its latent chunks and
 //     its RoPE share, loaded with a 16- or 32-column box swizzled to 32 or 64
 //     bytes), freed as soon as the page's score MMA completes;
@@ -56,7 +53,7 @@
 //     P*V, freed by P*V.  The second read is an L2 hit (the first was a few
 //     microseconds earlier), so HBM still sees every byte once;
 //   the RoPE part of the Q slice (SS MMA operand, swizzled like the page's
-//     RoPE share), the fp16 identity matrix, and the 16 KB P tile;
+//     RoPE share) and the 16 KB P tile (SS P*V operand);
 //   two 1 KB slots of half-row maxima for the finishers' pair exchange
 //     (a segment's row sums borrow the idle one).
 // Segment metadata and page ids are loaded a step ahead so no global load
@@ -64,15 +61,13 @@
 //
 // Warp roles (512 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
 // allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
-// exchange-MMA and P*V-MMA issuer (it polls the inputs of both streams and
-// issues whichever is ready, so neither waits on the other), all
-// warp-uniform with one elected lane issuing; warps 4-7 = sender (reads each page's own partial score from TMEM,
-// ships it to the peer, loads each segment's Q slice), warps 8-11 and 12-15 =
-// the two finisher halves (keys 0-31 and 32-63 of every row: softmax, P, and
+// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-7 =
+// sender (reads each page's own partial score from TMEM, ships it to the
+// peer, loads each segment's Q slice), warps 8-11 and 12-15 = the two
+// finisher halves (keys 0-31 and 32-63 of every row: score, softmax, P, and
 // half of O in the epilogue); thread r of any of these owns row r = TMEM
 // lane r.  Two score buffers let the score MMA of page t+1 run while the
-// finishers work on page t.  Every wait is bounded (sm100::mbar_wait; warp
-// 3's poll loop gives up after 2^32 cycles without progress).
+// finishers work on page t.  Every wait is bounded (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -94,25 +89,24 @@ constexpr int SG_BYTES = ROPE_OFF + KT * MAX_ROPE * 2;
 constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
 constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
 constexpr int QR_BYTES = 128 * MAX_ROPE * 2;  // the RoPE part of the Q slice
-constexpr int ID_BYTES = KT * KT * 2;         // 64 x 64 fp16 identity
 constexpr int P_BYTES = 128 * KT * 2;         // P tile: 128 rows x 64 keys bf16
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384, TM_COLS = 512;
 
 // The exchange buffers and the credit barriers sit at the same offsets in
-// both CTAs (the peer addresses them through mapa / a commit multicast).
+// both CTAs (the peer addresses them through mapa).
 constexpr int OFF_X = 0;
-constexpr int OFF_SG = OFF_X + XBUF * X_BYTES;
+constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
+constexpr int OFF_SG = OFF_XS + X_BYTES;
 constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
 constexpr int OFF_QR = OFF_VG + VGROUPS * VG_BYTES;
-constexpr int OFF_ID = OFF_QR + QR_BYTES;
-constexpr int OFF_P = OFF_ID + ID_BYTES;
+constexpr int OFF_P = OFF_QR + QR_BYTES;
 constexpr int OFF_MH = OFF_P + P_BYTES;           // half-row maxima [2][2][128] fp32 (sums reuse a slot)
 constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * XBUF + 2 * SGROUPS + 2 * VGROUPS + 2 + 2 + 2 + 2 + 1 + 1 + 3 + 4;
+constexpr int NUM_BARS = 2 * XBUF + 2 * SGROUPS + 2 * VGROUPS + 2 + 2 + 1 + 1 + 3 + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-static_assert(OFF_SG % 1024 == 0 && OFF_VG % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_ID % 1024 == 0 &&
-                  OFF_P % 1024 == 0 && SG_BYTES % 1024 == 0,
+static_assert(OFF_SG % 1024 == 0 && OFF_VG % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_P % 1024 == 0 &&
+                  SG_BYTES % 1024 == 0,
               "swizzled operands need 1024-byte aligned tiles");
 // No slack for aligning the base: the kernel has no static shared memory, so
 // its dynamic block starts on a 1024-byte boundary (the kernel checks this
@@ -155,19 +149,21 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// Asynchronous 16-byte store into a peer CTA's shared memory that completes
-// as 16 transaction bytes on the peer's mbarrier `bar_cluster_addr`.
-__device__ __forceinline__ void st_async_peer(uint32_t dst_cluster_addr, uint4 v, uint32_t bar_cluster_addr) {
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
+// a peer CTA's, completing as transaction bytes on the peer's mbarrier
+// `bar_cluster_addr`.  One copy carries what would otherwise be many small
+// remote stores, each with its own transaction-count update at the peer.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster_addr, uint32_t src_smem, uint32_t bytes,
+                                                  uint32_t bar_cluster_addr) {
   asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           dst_cluster_addr),
-      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
+      "r"(src_smem), "r"(bytes), "r"(bar_cluster_addr)
       : "memory");
 }
-// Asks L2 to fetch `bytes` (a multiple of 16) from global memory ahead of use.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the sources of this thread's committed bulk copies have been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Arrives once on the mbarrier at the same shared-memory offset in every CTA
 // of `cta_mask` when every tcgen05 operation this thread issued has completed.
 __device__ __forceinline__ void tc_commit_to(uint64_t* bar, uint16_t cta_mask) {
@@ -177,6 +173,10 @@ __device__ __forceinline__ void tc_commit_to(uint64_t* bar, uint16_t cta_mask) {
       "h"(cta_mask)
       : "memory");
 }
+// Asks L2 to fetch `bytes` (a multiple of 16) from global memory ahead of use.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 // Partial scores travel between the CTAs as fp16 pairs, saturated at
 // +-65504 (one conversion per pair).
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -184,18 +184,24 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
   return u;
 }
-// Instruction descriptor, kind::f16 with fp16 A and B (the exchanged
-// partials against the identity), fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// Exact fp16 pair -> two floats with integer work and one multiply per value
+// (no conversion-pipe work): the 15 bits below a half's sign, moved to an
+// fp32's exponent and significand positions, are its value times 2^-112
+// (subnormal halves included, as fp32 subnormals); the sign moves over.
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+  const float lo = __uint_as_float((u << 13) & 0x0fffe000u) * 0x1p112f;
+  const float hi = __uint_as_float((u >> 3) & 0x0fffe000u) * 0x1p112f;
+  return make_float2(__uint_as_float(__float_as_uint(lo) | ((u << 16) & 0x80000000u)),
+                     __uint_as_float(__float_as_uint(hi) | (u & 0x80000000u)));
 }
 
-// Byte offset, in an exchange tile (and in the P tile), of 16-byte piece u
+// Byte offset, in an exchange tile and in the P tile, of 16-byte piece u
 // (0..7) of row r's 64 16-bit values: row r at r * 128, piece u at
 // (u ^ (r & 7)) * 16.  This is the 128-byte-swizzled K-major operand layout
-// (8-row groups of 1 KB), so a received tile is the A operand of the exchange
-// MMA as it lands, and the eight rows a quarter-warp writes at once fall in
-// eight bank groups.
+// (8-row groups of 1 KB) the P*V MMA reads P in; each warp's 32 rows are one
+// contiguous 4 KB block (one bulk copy), and the eight rows a quarter-warp
+// touches at once fall in eight bank groups.
+constexpr int X_WARP_BYTES = 32 * KT * 2;
 __device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 // Byte offset of 16-byte piece u of row r in the RoPE part of the Q slice,
 // rows of rw * 2 bytes swizzled to that width (64-byte rows: piece ^ row
@@ -214,15 +220,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
-  uint64_t* x_free = x_full + XBUF;      // [XBUF] the peer has consumed what this CTA sent into its buffer
+  uint64_t* x_free = x_full + XBUF;      // [XBUF] the peer has consumed what this CTA sent
   uint64_t* sg_full = x_free + XBUF;     // [SGROUPS]
   uint64_t* sg_empty = sg_full + SGROUPS;
   uint64_t* vg_full = sg_empty + SGROUPS;  // [VGROUPS]
   uint64_t* vg_empty = vg_full + VGROUPS;
   uint64_t* s_full = vg_empty + VGROUPS;   // [2] own partial score in buffer b
-  uint64_t* s_read = s_full + 2;           // [2] the sender has read the own partial in buffer b
-  uint64_t* s_total = s_read + 2;          // [2] the peer's partial has been added into buffer b
-  uint64_t* s_free = s_total + 2;          // [2] the finishers have read buffer b
+  uint64_t* s_free = s_full + 2;           // [2] the sender and the finishers have read buffer b
   uint64_t* p_ready = s_free + 2;          // P of the current page is in the P tile
   uint64_t* pv_done = p_ready + 1;         // P*V of the current page has completed
   uint64_t* q_ready = pv_done + 1;
@@ -248,7 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (tid == 32) {
     for (int i = 0; i < XBUF; ++i) {
       mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
-      mbar_init(&x_free[i], 1);  // the peer's commit
+      mbar_init(&x_free[i], 1);  // the peer's P*V commit
     }
     for (int i = 0; i < SGROUPS; ++i) {
       mbar_init(&sg_full[i], 1);
@@ -260,9 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_read[i], 128);  // sender
-      mbar_init(&s_total[i], 1);
-      mbar_init(&s_free[i], 256);  // finishers
+      mbar_init(&s_free[i], 384);  // sender + finishers
     }
     mbar_init(p_ready, 256);  // finishers
     mbar_init(pv_done, 1);
@@ -272,18 +274,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
     *abort_flag = 0;
     mbar_fence_init();
-  }
-  // The 64 x 64 fp16 identity (B operand of the exchange MMA), K-major with
-  // the 128-byte swizzle: row n holds 1.0 at column n.
-  {
-    const int n = tid >> 3, u = tid & 7;  // 512 threads: one 16-byte piece each
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if ((n >> 3) == u) {
-      uint32_t* e = reinterpret_cast<uint32_t*>(&v);
-      e[(n & 7) >> 1] = (n & 1) ? 0x3C000000u : 0x00003C00u;
-    }
-    *reinterpret_cast<uint4*>(smem + OFF_ID + n * 128 + ((u ^ (n & 7)) << 4)) = v;
-    fence_proxy_async_smem();
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, TM_COLS);
@@ -357,8 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------- score-MMA issuer
-    // Page t's partial score goes into buffer t & 1, free once the finishers
-    // have read page t - 2's scores from it.
+    // Page t's partial score goes into buffer t & 1, free once the sender and
+    // the finishers have read page t - 2's scores from it.
     const uint32_t tS = tbase + TM_S, tQ = tbase + TM_Q;
     const uint32_t sSG = smem_u32(smem + OFF_SG), sQR = smem_u32(smem + OFF_QR);
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);
@@ -401,85 +391,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     __syncwarp();
     mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
   } else if (warp == 3) {
-    // ---------------------------------------- exchange-MMA and P*V issuer
-    // Two in-order streams: the exchange MMA of page t (S_t += X_peer,t * I,
-    // once the sender has read the own partial and the peer's has landed;
-    // its completion also hands the exchange buffer back to the peer) and
-    // P*V of page t (once the finishers have written P_t).  The warp polls
-    // the inputs of both and issues whichever is ready, so a late peer copy
-    // never holds back P*V and the reverse.
-    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O;
-    const uint32_t sX = smem_u32(smem + OFF_X), sID = smem_u32(smem + OFF_ID), sVG = smem_u32(smem + OFF_VG);
-    const uint32_t sP = smem_u32(smem + OFF_P);
-    const uint32_t idX = idesc_f16(128, KT), idPV = idesc_bf16(128, dh, 0, 1);
-    int total = 0;  // pages of this worker
-    for (int s = seg_lo + (tid & 31); s < seg_hi; s += 32) total += segs[s].t_hi - segs[s].t_lo;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-    uint32_t xt = 0, pt = 0;       // next page of each stream
-    int si = seg_lo, pi = 0, seg_k = 0;  // P*V stream: segment, page in it, segment count
-    int seg_n = seg_lo < seg_hi ? segs[seg_lo].t_hi - segs[seg_lo].t_lo : 0;
-    // Progress deadline in SM cycles (clock64 is a register read; the global
-    // timer is far slower to read, which would delay every poll): 2^32 cycles,
-    // 2-4 s at the clocks this part runs at.
-    long long t_prog = clock64();
-    while ((int)pt < total) {
-      bool prog = false;
-      if ((int)xt < total) {
-        const uint32_t b = xt & 1, xb = xt % XBUF;
-        if (mbar_try_wait_warp(&s_read[b], (xt >> 1) & 1) && mbar_try_wait_warp(&x_full[xb], (xt / XBUF) & 1)) {
-          fence_proxy_async_smem();  // the peer's stores, now visible here, to the MMA's proxy
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int k = 0; k < KT / 16; ++k)
-              mma_ss(tS + b * KT, sdesc_sw128(sX + xb * X_BYTES + k * 32, 16, 1024),
-                     sdesc_sw128(sID + k * 32, 16, 1024), idX, 1u);
-            tc_commit(&s_total[b]);
-            tc_commit_to(&x_free[xb], (uint16_t)(1u << peer));  // the peer may refill buffer xb
-          }
-          __syncwarp();
-          ++xt;
-          prog = true;
-        }
-      }
-      if (pt < xt) {
-        const uint32_t vs = pt % VGROUPS;
-        if (mbar_try_wait_warp(p_ready, pt & 1) &&
-            (pi != 0 || seg_k == 0 || mbar_try_wait_warp(o_free, (seg_k - 1) & 1)) &&
-            mbar_try_wait_warp(&vg_full[vs], (pt / VGROUPS) & 1)) {
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < KT / 16; ++kk)
-              mma_ss(tO, sdesc_sw128(sP + kk * 32, 16, 1024),
-                     sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
-                     (pi == 0 && kk == 0) ? 0u : 1u);
-            tc_commit(pv_done);
-            tc_commit(&vg_empty[vs]);
-          }
-          __syncwarp();
-          ++pt;
-          if (++pi == seg_n) {
-            pi = 0;
-            ++seg_k;
-            if (++si < seg_hi) seg_n = segs[si].t_hi - segs[si].t_lo;
-          }
-          prog = true;
-        }
-      }
-      if (prog) {
-        t_prog = clock64();
-      } else if (*abort_flag) {
-        break;
-      } else if (clock64() - t_prog > (1ll << 32)) {
+    // ------------------------------------------------------ P*V issuer
+    const uint32_t tO = tbase + TM_O;
+    const uint32_t sVG = smem_u32(smem + OFF_VG), sP = smem_u32(smem + OFF_P);
+    const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
+    uint32_t tg = 0, seg_k = 0;
+    bool ok = true;
+    Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
+    for (int si = seg_lo; si < seg_hi && ok; ++si) {
+      const Seg g = gn;
+      if (si + 1 < seg_hi) gn = segs[si + 1];
+      const int n = g.t_hi - g.t_lo;
+      for (int i = 0; i < n; ++i, ++tg) {
+        if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
+        if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
+        const uint32_t vs = tg % VGROUPS;
+        if (!(ok = mbar_wait_warp(&vg_full[vs], (tg / VGROUPS) & 1, abort_flag, a.err))) break;
+        tc_fence_after();
         if (elect_one()) {
-          *abort_flag = 1;
-          flag_error(a.err, kErrTimeout);
+#pragma unroll
+          for (int kk = 0; kk < KT / 16; ++kk)
+            mma_ss(tO, sdesc_sw128(sP + kk * 32, 16, 1024),
+                   sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
+                   (i == 0 && kk == 0) ? 0u : 1u);
+          tc_commit(pv_done);
+          tc_commit(&vg_empty[vs]);
+          // The finishers read exchange buffer tg % XBUF before P_tg was
+          // ready: hand it back to the peer's sender.
+          tc_commit_to(&x_free[tg % XBUF], (uint16_t)(1u << peer));
         }
         __syncwarp();
-        break;
       }
+      ++seg_k;
     }
     if (elect_one()) tc_commit(final_bar);
     __syncwarp();
@@ -501,9 +444,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (sender) {
       // Reads each page's own partial score (all 64 keys of its row) from
-      // TMEM, packs it to fp16 and stores it straight into the peer's
-      // exchange buffer; also loads each segment's Q slice.
+      // TMEM, packs it to fp16, stages it and ships it to the peer with one
+      // bulk copy per warp; also loads each segment's Q slice.
       uint8_t* sQR = smem + OFF_QR;
+      uint8_t* sXS = smem + OFF_XS;
       const uint32_t peer_x = map_peer(smem_u32(smem + OFF_X), peer);
       const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
       const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
@@ -579,19 +523,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
           }
           tc_fence_before();
-          mbar_arrive(&s_read[b]);
+          mbar_arrive(&s_free[b]);
           // The segment's scores are all read after its last page, so the next
           // segment's Q may replace this one's.
           if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
-          // The peer's partial of this page will land in exchange buffer xb.
-          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
-          // Buffer xb of the peer is free once its exchange MMA of page
-          // tg - XBUF has completed.
-          if (tg >= XBUF && !(ok = wait_all(&x_free[xb], ((tg / XBUF) - 1) & 1))) break;
+          // The staging block is reused once the copy engine has read it.
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            st_async_peer(peer_x + xb * X_BYTES + x_off(r, u),
-                          make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]), peer_xbar + xb * 8);
+            *reinterpret_cast<uint4*>(sXS + x_off(r, u)) =
+                make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]);
+          fence_proxy_async_smem();  // the copy engine reads what the threads wrote
+          // The peer's partial of this page will land in exchange buffer xb.
+          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
+          // Buffer xb of the peer is free once its finishers have read page
+          // tg - XBUF from it.
+          if (tg >= XBUF && !(ok = wait_all(&x_free[xb], ((tg / XBUF) - 1) & 1))) break;
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t blk = (uint32_t)((warp & 3) * X_WARP_BYTES);
+            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, X_WARP_BYTES, peer_xbar + xb * 8);
+            bulk_commit();
+          }
         }
         g_cur = g_nxt;
         if (si + 2 < seg_hi) g_nxt = segs[si + 2];
@@ -602,6 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (ok)
         for (uint32_t pg = tg > (uint32_t)XBUF ? tg - XBUF : 0; pg < tg; ++pg)
           if (!wait_all(&x_free[pg % XBUF], (pg / XBUF) & 1)) break;
+      if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
     } else {
       // Two finisher warpgroups: half h owns keys [32h, 32h + 32) of every
       // row and half of O's columns; the two threads of a row (their warps
@@ -621,6 +576,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
       uint8_t* sV = smem + OFF_VG;
       uint8_t* sPt = smem + OFF_P;
+      const uint8_t* sX = smem + OFF_X;
       float m_used = -INFINITY, l = 0.f;
       uint32_t tg = 0;
       for (int si = seg_lo; si < seg_hi && ok; ++si) {
@@ -629,8 +585,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int i = 0; i < n; ++i, ++tg) {
           const int t = g.t_lo + i;
           const uint32_t b = tg & 1;
-          // Own + peer partial, summed by the exchange MMA.
-          if (!(ok = wait_all(&s_total[b], (tg >> 1) & 1))) break;
+          // This CTA's exact partial from TMEM (the buffer is released at
+          // once), then the peer's fp16 partial from the exchange buffer.
+          if (!(ok = wait_all(&s_full[b], (tg >> 1) & 1))) break;
           tc_fence_after();
           float s[32];
           {
@@ -642,6 +599,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           tc_fence_before();
           mbar_arrive(&s_free[b]);  // the score MMA of page tg + 2 may overwrite it
+          const uint32_t xb = tg % XBUF;
+          if (!(ok = wait_all(&x_full[xb], (tg / XBUF) & 1))) break;
+          {
+            uint4 pv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pv[u] = *reinterpret_cast<const uint4*>(sX + xb * X_BYTES + x_off(r, 4 * h + u));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t pw[4] = {pv[u].x, pv[u].y, pv[u].z, pv[u].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 y = unpack_f16x2(pw[e]);
+                s[8 * u + 2 * e] += y.x;
+                s[8 * u + 2 * e + 1] += y.y;
+              }
+            }
+          }
           const int valid_all = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
           const int valid = valid_all - 32 * h;             // valid keys among this half's 32
           if (valid < 32) {
@@ -682,9 +657,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             float ps[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+            // The row sum adds the fp32 weights (not their bf16 roundings: the
+            // difference is random, 2^-9 relative per key, and unpacking the
+            // rounded pairs would cost two more instructions per pair).
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              pk[u] = pack_bf16(fast_exp2(s[2 * u] - m_used), fast_exp2(s[2 * u + 1] - m_used), ps[u & 7]);
+            for (int u = 0; u < 16; ++u) {
+              const float e0 = fast_exp2(s[2 * u] - m_used), e1 = fast_exp2(s[2 * u + 1] - m_used);
+              ps[u & 7] += e0 + e1;
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
+              pk[u] = *reinterpret_cast<uint32_t*>(&v2);
+            }
 #pragma unroll
             for (int w2 = 4; w2 >= 1; w2 >>= 1)
 #pragma unroll

@@ -46,8 +46,9 @@ struct EpiStore {
   }
 };
 
-// Append: columns [0, d_c) are the latent, [d_c, d_c + d_r) the position key,
-// rotated by the token's position, then the row goes to its cache slot.
+// Append: columns [0, d_c) are the latent, [d_c, d_cr) the position key (one
+// shared key of d_r, or one per head), every d_r-wide key rotated by the
+// token's position, then the row goes to its cache slot.
 // Without seq_idx/pos (prefill), row m is token m % prefill_S of sequence
 // m / prefill_S.
 template <typename OutT>
@@ -59,6 +60,7 @@ struct EpiAppend {
   const int32_t* page_table;
   double theta[32];        // RoPE frequencies
   int max_pages, num_pages, page_size, d_c, d_cr, n_seq;
+  int d_r;                 // RoPE-key width: columns [d_c, d_cr) are one key or n_h keys of d_r each
   int* err;
   OutT* dense;             // optional: every row also at dense[m * d_cr] (token order), else null
   __device__ void operator()(int, int m, int n, float v0, float v1) const {
@@ -79,7 +81,7 @@ struct EpiAppend {
       flag_error(err, kErrBounds);
       return;
     }
-    if (n >= d_c) rope_rotate_pair(v0, v1, p, theta[(n - d_c) >> 1]);
+    if (n >= d_c) rope_rotate_pair(v0, v1, p, theta[((n - d_c) % d_r) >> 1]);
     store_pair(cache + ((long long)page * page_size + p % page_size) * d_cr + n, v0, v1);
     if (dense) store_pair(dense + (long long)m * d_cr + n, v0, v1);
   }
@@ -108,7 +110,7 @@ struct EpiAppend {
     for (int i = 0; i < 8; ++i) w[i] = v[i];
     if (n0 >= d_c) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) rope_rotate_pair(w[2 * i], w[2 * i + 1], p, theta[((n0 - d_c) >> 1) + i]);
+      for (int i = 0; i < 4; ++i) rope_rotate_pair(w[2 * i], w[2 * i + 1], p, theta[(((n0 - d_c) % d_r) >> 1) + i]);
     }
     mla::store8(cache + ((long long)page * page_size + p % page_size) * d_cr + n0, w);
     if (dense) mla::store8(dense + (long long)m * d_cr + n0, w);

@@ -29,7 +29,7 @@ struct mla_weights {
   mla_dims d;
   float scale;         // softmax scale actually used
   size_t esz;          // element size of the path (4 or 2)
-  void* dkr;           // [d_c + d_r][d_model]
+  void* dkr;           // [d_cr][d_model]: W_DKV then W_KR (d_r rows, or n_h * d_r per head)
   void* dq;            // [d_cq][d_model] or null
   void* uqr;           // [n_h*(d_h + d_r)][d_in]
   void* ukt;           // [n_h][d_c][d_h]
@@ -106,8 +106,16 @@ cudaError_t set_smem_once(F* fn, size_t bytes) {
   return cudaSuccess;
 }
 
+// Cache row width: the latent, then one shared RoPE key or one per head.
+int cache_row(const mla_dims& d) { return d.d_c + (d.rope_key_per_head ? d.n_h : 1) * d.d_r; }
+
+// Rows of a cache row that the CUDA-core attention kernel stages per key
+// (shared memory: 32 keys plus up to 16 heads' queries, fp32).
+constexpr int kSimtMaxRow = 1024;
+
 mla_status check_dims(const mla_dims* d) {
   if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->rope_key_per_head != 0 && d->rope_key_per_head != 1) return MLA_ERR_INVALID_ARG;
   if (d->n_h <= 0 || d->d_h <= 0 || d->d_v <= 0 || d->d_c <= 0 || d->d_r <= 0 || d->d_model <= 0 ||
       d->d_cq < 0 || d->page_size <= 0 || !(d->rope_base > 0.f) || d->softmax_scale < 0.f)
     return MLA_ERR_INVALID_ARG;
@@ -120,10 +128,13 @@ mla_status check_dims(const mla_dims* d) {
     // two halves of whole 64-column chunks; a cache row is at most nine chunks.
     if (d->d_h % 8 || d->d_v % 8 || d->d_c % 128 || d->d_r % 16 || d->d_model % 8 || d->d_cq % 8)
       return MLA_ERR_UNSUPPORTED;
-    if (d->d_c > 512 || d->d_c + d->d_r > 576) return MLA_ERR_UNSUPPORTED;
+    if (d->d_c > 512 || (!d->rope_key_per_head && d->d_c + d->d_r > 576)) return MLA_ERR_UNSUPPORTED;
   } else {
     if (d->d_c > 512) return MLA_ERR_UNSUPPORTED;
   }
+  // Per-head RoPE keys run on the CUDA-core attention kernel, which stages
+  // whole cache rows.
+  if (d->rope_key_per_head && cache_row(*d) > kSimtMaxRow) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -137,7 +148,7 @@ WeightLayout weight_layout(const mla_dims& d) {
   const size_t e = esize(d);
   WeightLayout L{};
   size_t o = 0;
-  L.dkr = o; o = align_up(o + e * (d.d_c + d.d_r) * d.d_model, 256);
+  L.dkr = o; o = align_up(o + e * (size_t)cache_row(d) * d.d_model, 256);
   L.dq = o;  o = align_up(o + e * (size_t)d.d_cq * d.d_model, 256);
   L.uqr = o; o = align_up(o + e * (size_t)d.n_h * (d.d_h + d.d_r) * d_in(d), 256);
   L.ukt = o; o = align_up(o + e * (size_t)d.n_h * d.d_c * d.d_h, 256);
@@ -369,10 +380,11 @@ mla_status append_impl(const mla_weights* w, const void* h, const int32_t* seq_i
   epi.num_pages = num_pages;
   epi.page_size = d.page_size;
   epi.d_c = d.d_c;
-  epi.d_cr = d.d_c + d.d_r;
+  epi.d_cr = cache_row(d);
+  epi.d_r = d.d_r;
   epi.n_seq = n_seq;
   epi.err = at<int>(ws, P.hdr);
-  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, d.d_c + d.d_r, d.d_model, 1, epi,
+  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, cache_row(d), d.d_model, 1, epi,
                              ws, P, st));
 }
 
@@ -390,7 +402,8 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
                        const void* cache, float* out, int R, int max_kv_len, void* ws, const Plan& P,
                        cudaStream_t st, const CpOut* cp = nullptr) {
   const mla_dims& d = w->d;
-  const int d_cr = d.d_c + d.d_r;
+  const int q_row = d.d_c + d.d_r;  // a Q_abs row: [q~ | q_R]
+  const int d_cr = cache_row(d);    // a cache row: [c | k_R] (one key or n_h)
   const int din = d_in(d);
   int* err = at<int>(ws, P.hdr);
   cudaError_t e;
@@ -411,7 +424,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     epi.kv_len = kv_len;
     epi.uniform_kv_len = uniform_kv_len;
     for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
-    epi.n_h = d.n_h; epi.d_h = d.d_h; epi.d_r = d.d_r; epi.d_c = d.d_c; epi.d_cr = d_cr;
+    epi.n_h = d.n_h; epi.d_h = d.d_h; epi.d_r = d.d_r; epi.d_c = d.d_c; epi.d_cr = q_row;
     epi.qabs_rows = P.qrows; epi.n_q = n_q; epi.prefill_S = prefill_S;
     epi.qr_scale = qscale;
     if ((e = gemm<T>(src, din, 0, w->uqr, din, 0, R, d.n_h * (d.d_h + d.d_r), din, 1, epi, ws, P, st)))
@@ -419,7 +432,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   }
   // (3) absorption q~_h = W_UK,h^T q_C,h, scaled.
   {
-    EpiStore<T> epi{at<T>(ws, P.qabs), (long long)P.qrows * d_cr, d_cr, qscale};
+    EpiStore<T> epi{at<T>(ws, P.qabs), (long long)P.qrows * q_row, q_row, qscale};
     if ((e = gemm<T>(at<T>(ws, P.qc), (long long)d.n_h * d.d_h, d.d_h, w->ukt, d.d_h, (long long)d.d_c * d.d_h,
                      R, d.d_c, d.d_h, d.n_h, epi, ws, P, st)))
       return cuda_status(e);
@@ -436,6 +449,8 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   aa.num_pages = num_pages;
   aa.page_size = d.page_size;
   aa.n_h = d.n_h; aa.d_c = d.d_c; aa.d_r = d.d_r; aa.d_cr = d_cr;
+  aa.q_row = q_row;
+  aa.rope_per_head = d.rope_key_per_head;
   aa.kv_len = kv_len; aa.uniform_kv_len = uniform_kv_len; aa.n_q = n_q; aa.max_kv_len = max_kv_len;
   aa.sched = S;
   aa.part_o = at<float>(ws, P.part_o);
@@ -443,7 +458,10 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   aa.obar = at<T>(ws, P.obar);
   aa.err = err;
 
-  constexpr bool kTensorCores = sizeof(T) == 2;
+  // bf16 with one shared RoPE key runs on the tensor cores; per-head RoPE
+  // keys (whose position term is a per-head contraction, not one dense
+  // product over the shared row) and fp32 run on the CUDA cores.
+  const bool kTensorCores = sizeof(T) == 2 && !d.rope_key_per_head;
   // fp32: heads per CTA a power of two so that 256 threads split evenly.
   int HG = 16;
   while (HG > d.n_h) HG >>= 1;
@@ -464,7 +482,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (5) attention on the latent cache, (6) combine of split row blocks.
-  if constexpr (kTensorCores) {
+  if (kTensorCores) {
     CUtensorMap map;
     const long long rows = (long long)num_pages * d.page_size;
     CUtensorMap rmap16, rmap32;
@@ -534,7 +552,7 @@ MatPlan make_mat_plan(const mla_dims& d, int T) {
 // Dimensions the materialised kernel takes: bf16, a 64-wide RoPE key, and
 // head widths that are whole 64-column chunks of at most 128.
 bool mat_supported(const mla_dims& d) {
-  return d.dtype == MLA_BF16 && d.d_r == attn_mha::DR && (d.d_h == 64 || d.d_h == 128) &&
+  return d.dtype == MLA_BF16 && !d.rope_key_per_head && d.d_r == attn_mha::DR && (d.d_h == 64 || d.d_h == 128) &&
          (d.d_v == 64 || d.d_v == 128);
 }
 
@@ -558,6 +576,7 @@ mla_status prefill_mat_impl(const mla_weights* w, const void* h, const int32_t* 
     epi.page_size = d.page_size;
     epi.d_c = d.d_c;
     epi.d_cr = d_cr;
+    epi.d_r = d.d_r;
     epi.n_seq = B;
     epi.err = at<int>(ws, P.hdr);
     epi.dense = at<T>(ws, M.dense);
@@ -708,7 +727,7 @@ mla_status mla_absorb_weights(const mla_dims* dims, const void* W_DKV, const voi
   g_launches = 0;
   cudaError_t err;
   // Stacked [W_DKV; W_KR] and [W_UQ; W_QR]: plain contiguous copies.
-  size_t n1 = e * (size_t)d.d_c * d.d_model, n2 = e * (size_t)d.d_r * d.d_model;
+  size_t n1 = e * (size_t)d.d_c * d.d_model, n2 = e * (size_t)(cache_row(d) - d.d_c) * d.d_model;
   if ((err = cudaMemcpyAsync(base + L.dkr, W_DKV, n1, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
   if ((err = cudaMemcpyAsync(base + L.dkr + n1, W_KR, n2, cudaMemcpyDeviceToDevice, stream))) return cuda_status(err);
   if (d.d_cq > 0 &&
@@ -809,7 +828,8 @@ mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_l
 }
 
 size_t mla_decode_cp_workspace_bytes(const mla_dims* dims, int B, int n_q) {
-  if (check_dims(dims) != MLA_OK || dims->dtype != MLA_BF16 || B <= 0 || n_q <= 0) return 0;
+  if (check_dims(dims) != MLA_OK || dims->dtype != MLA_BF16 || dims->rope_key_per_head || B <= 0 || n_q <= 0)
+    return 0;
   return make_plan(*dims, B * n_q, true, true).total;
 }
 
@@ -820,7 +840,7 @@ mla_status mla_decode_cp_partial(const mla_weights* w, const void* h_q, const in
                                  size_t workspace_bytes, cudaStream_t stream) {
   if (!w || B <= 0 || n_q <= 0 || max_kv_len < n_q || max_pages <= 0 || num_pages <= 0)
     return MLA_ERR_INVALID_ARG;
-  if (w->d.dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if (w->d.dtype != MLA_BF16 || w->d.rope_key_per_head) return MLA_ERR_UNSUPPORTED;
   if (!h_q || !kv_len || !window_start || !window_count || !page_table || !cache || !obar_out || !lse_out ||
       !workspace)
     return MLA_ERR_INVALID_ARG;
@@ -841,7 +861,7 @@ mla_status mla_decode_cp_combine(const mla_weights* w, int n_ranks, const void* 
                                  const float* lse_parts, float* out, int B, int n_q, void* workspace,
                                  size_t workspace_bytes, cudaStream_t stream) {
   if (!w || n_ranks <= 0 || B <= 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
-  if (w->d.dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if (w->d.dtype != MLA_BF16 || w->d.rope_key_per_head) return MLA_ERR_UNSUPPORTED;
   if (!obar_parts || !lse_parts || !out || !workspace) return MLA_ERR_INVALID_ARG;
   if (!aligned(workspace, 256) || !aligned(obar_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16))
     return MLA_ERR_INVALID_ARG;
@@ -1012,10 +1032,11 @@ mla_status append_noalloc_impl(const mla_weights* w, const void* h, const int32_
   epi.num_pages = num_pages;
   epi.page_size = d.page_size;
   epi.d_c = d.d_c;
-  epi.d_cr = d.d_c + d.d_r;
+  epi.d_cr = cache_row(d);
+  epi.d_r = d.d_r;
   epi.n_seq = num_seqs;
   epi.err = device_error ? reinterpret_cast<int*>(device_error) : at<int>(scratch, P.hdr);
-  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, d.d_c + d.d_r, d.d_model, 1, epi, scratch,
+  return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, cache_row(d), d.d_model, 1, epi, scratch,
                              P, st, kNoAllocTileSplits));
 }
 

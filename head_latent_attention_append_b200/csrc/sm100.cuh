@@ -72,17 +72,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // *abort and returns false, so no thread can spin forever.
 // With honor_abort = false the wait ignores *abort (used to drain work that is
 // already in flight before the CTA exits).
+// The loop polls with the plain try_wait (which itself waits a short,
+// hardware-chosen time): a long suspend-time hint measured ~0.4 us between a
+// phase completing and a sleeping waiter resuming.  The global timer, slow to
+// read, is checked every 64 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
                                           uint64_t limit_ns = 2000000000ull, bool honor_abort = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
-    if (honor_abort && *abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      flag_error(err, kErrTimeout);
-      return false;
+  for (uint32_t k = 1;; ++k) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((k & 63) == 0) {
+      if (honor_abort && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        flag_error(err, kErrTimeout);
+        return false;
+      }
     }
   }
 }

@@ -41,12 +41,13 @@ class Dims(ctypes.Structure):
     _fields_ = [("n_h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_v", ctypes.c_int), ("d_c", ctypes.c_int),
                 ("d_r", ctypes.c_int), ("d_model", ctypes.c_int), ("d_cq", ctypes.c_int),
                 ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float), ("page_size", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("rope_key_per_head", ctypes.c_int)]
 
 
 def make_dims(n_h, d_h, d_v, d_c, d_r, d_model, d_cq=0, rope_base=10000.0, softmax_scale=0.0,
-              page_size=64, dtype=BF16) -> Dims:
-    return Dims(n_h, d_h, d_v, d_c, d_r, d_model, d_cq, rope_base, softmax_scale, page_size, dtype)
+              page_size=64, dtype=BF16, rope_key_per_head=0) -> Dims:
+    return Dims(n_h, d_h, d_v, d_c, d_r, d_model, d_cq, rope_base, softmax_scale, page_size, dtype,
+                int(rope_key_per_head))
 
 
 def _load():

@@ -49,18 +49,21 @@ class Workload:
     max_cached: int = 0     # ragged: lengths drawn from U{1..max_cached}
     rope_base: float = 10000.0
     materialised: bool = False  # prefill through expanded per-head keys and values
+    rope_per_head: bool = False  # one RoPE key per head in every cache row instead of one shared
 
     @property
     def d_cr(self) -> int:
-        return self.d_c + self.d_r
+        """Cache row width: the latent, then one shared RoPE key or n_h of them."""
+        return self.d_c + (self.n_h if self.rope_per_head else 1) * self.d_r
 
     def flops_per_pair(self) -> int:
         """Algorithmic flops per causal (query, key) pair, all heads: the
-        absorbed form scores over d_c + d_r columns and sums d_c latent
-        columns; the materialised form scores over d_h + d_r and sums d_v."""
+        absorbed form scores each head over d_c + d_r columns (its own RoPE key
+        in the per-head layout) and sums d_c latent columns; the materialised
+        form scores over d_h + d_r and sums d_v."""
         if self.materialised:
             return self.n_h * (2 * (self.d_h + self.d_r) + 2 * self.d_v)
-        return self.n_h * (2 * self.d_cr + 2 * self.d_c)
+        return self.n_h * (2 * (self.d_c + self.d_r) + 2 * self.d_c)
 
 
 WORKLOADS = {
@@ -74,6 +77,9 @@ WORKLOADS = {
         # Multi-token (speculative-style) decode: 4 new tokens per sequence over ragged histories.
         Workload("dsv2_spec4_decode", 6, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "decode", 64, 4, 0,
                  ragged=True, max_cached=32768),
+        # Config 2's model with one 32-dim RoPE key per head (cache row 256 + 16 x 32 = 768).
+        Workload("page_bf16_decode_rph", 8, 16, 128, 128, 256, 32, 2048, 0, "bf16", "decode", 8, 1, 4096,
+                 rope_per_head=True),
         # The causal prefill of config 4 (same seeds, same inputs) in the materialised form.
         Workload("dsv2_bf16_prefill_mat", 4, 128, 128, 128, 512, 64, 5120, 1536, "bf16", "prefill", 4, 4096, 0,
                  materialised=True),
@@ -120,7 +126,7 @@ def make_weights(wl: Workload, seed: int = BASE_SEED) -> HostWeights:
                        wl.dtype)
 
     W_DKV = draw(wl.d_c, wl.d_model)
-    W_KR = draw(wl.d_r, wl.d_model)
+    W_KR = draw(wl.d_r * (wl.n_h if wl.rope_per_head else 1), wl.d_model)
     W_DQ = draw(wl.d_cq, wl.d_model) if wl.d_cq > 0 else None
     W_UQ = draw(wl.n_h * wl.d_h, d_in)
     W_QR = draw(wl.n_h * wl.d_r, d_in)

@@ -20,7 +20,8 @@ TORCH_DTYPE = {"bf16": torch.bfloat16, "f32": torch.float32}
 
 def dims_of(wl: synth.Workload, softmax_scale: float = 0.0) -> mla.Dims:
     return mla.make_dims(wl.n_h, wl.d_h, wl.d_v, wl.d_c, wl.d_r, wl.d_model, wl.d_cq, wl.rope_base,
-                         softmax_scale, synth.PAGE_SIZE, mla.BF16 if wl.dtype == "bf16" else mla.F32)
+                         softmax_scale, synth.PAGE_SIZE, mla.BF16 if wl.dtype == "bf16" else mla.F32,
+                         wl.rope_per_head)
 
 
 def upload_weights(wl: synth.Workload, hw: synth.HostWeights, device) -> Dict[str, torch.Tensor]:

@@ -27,8 +27,9 @@
  *   - The library allocates no device memory.  Scratch space is the caller's
  *     `workspace`, sized by the *_workspace_bytes queries; the workspace of a
  *     call must not be used by another call that may run at the same time.
- *   - Cache layout: [num_pages, page_size, d_c + d_r]; row (page p, slot s)
- *     holds [c_t (d_c) | k_R,t (d_r)] for the token whose position is
+ *   - Cache layout: [num_pages, page_size, d_cr]; row (page p, slot s) holds
+ *     [c_t (d_c) | k_R,t (d_r)] (d_cr = d_c + d_r; with per-head RoPE keys
+ *     d_cr = d_c + n_h*d_r, see mla_dims) for the token whose position is
  *     j*page_size + s, where page_table[seq*max_pages + j] == p.
  *   - Weight orientation is column-vector, y = W x: W_DKV [d_c, d_model],
  *     W_KR [d_r, d_model], W_DQ [d_cq, d_model], W_UQ [n_h*d_h, d_in],
@@ -76,7 +77,21 @@ typedef struct {
   float softmax_scale;  /* 0 selects 1/sqrt(d_h + d_r) on both score terms   */
   int page_size;        /* tokens per cache page; this build supports 64     */
   mla_dtype dtype;      /* element type of weights, hidden states and cache  */
+  int rope_key_per_head; /* 0: one RoPE key shared by all heads (default);
+                            1: one d_r key per head (see below)              */
 } mla_dims;
+
+/* Per-head RoPE keys (rope_key_per_head = 1).  The 16-head example of "Multi-
+ * Head Latent Attention" (talalahmed), "A concrete size comparison", caches
+ * one d_r-dim position key per head instead of one shared key: W_KR is then
+ * [n_h*d_r, d_model] (rows h*d_r .. for head h), a cache row is
+ * [c_t (d_c) | k_R,0,t | ... | k_R,n_h-1,t] (d_c + n_h*d_r values, e.g.
+ * 256 + 16*32 = 768 for that example against 288 with a shared key), and head
+ * h's position term is q_R,h . k_R,h,t.  The position term is then a per-head
+ * contraction rather than part of one dense product over a shared row, so
+ * this layout runs on the CUDA-core attention kernel (fp32 and bf16) and
+ * needs d_c + n_h*d_r <= 1024; context-parallel decode and the materialised
+ * prefill return MLA_ERR_UNSUPPORTED for it. */
 
 /* Opaque host-side handle created by mla_absorb_weights.  It holds the
  * dimensions and pointers into the caller's `absorbed` device buffer. */

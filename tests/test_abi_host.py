@@ -58,6 +58,15 @@ def test_size_queries(mla):
     assert mla.decode_cp_workspace_bytes(d, 1024, 1) > mla.decode_workspace_bytes(d, 1024, 1, 8193)
     assert mla.decode_cp_workspace_bytes(dims3(mla, dtype=mla.F32), 4, 1) == 0
     assert mla.decode_cp_workspace_bytes(d, 0, 1) == 0
+    # Per-head RoPE keys: cache rows of d_c + n_h * d_r up to 1024 (the 16-head, 32-dim page example: 768);
+    # the absorbed weights hold n_h RoPE-key projections; no context-parallel or materialised path.
+    page = dict(n_h=16, d_h=128, d_v=128, d_c=256, d_r=32, d_model=2048, d_cq=0)
+    shared, per_head = dims3(mla, **page), dims3(mla, rope_key_per_head=1, **page)
+    assert mla.absorbed_weights_bytes(per_head) - mla.absorbed_weights_bytes(shared) >= 2 * 15 * 32 * 2048
+    assert mla.absorbed_weights_bytes(dims3(mla, rope_key_per_head=1)) == 0       # 512 + 128 * 64 > 1024
+    assert mla.absorbed_weights_bytes(dims3(mla, rope_key_per_head=2)) == 0
+    assert mla.decode_cp_workspace_bytes(per_head, 4, 1) == 0
+    assert mla.prefill_materialised_workspace_bytes(dims3(mla, rope_key_per_head=1, n_h=8), 2, 64) == 0
     # Materialised prefill: bf16, d_r = 64, d_h and d_v in {64, 128}; it holds the expanded K_C and V.
     assert mla.prefill_materialised_workspace_bytes(d, 4, 4096) >= 2 * 4 * 4096 * 128 * (128 + 128)
     assert mla.prefill_materialised_workspace_bytes(dims3(mla, d_r=32), 4, 4096) == 0
