@@ -32,7 +32,8 @@ struct AttnArgs {
   const int32_t* kv_len;
   int uniform_kv_len, n_q, max_kv_len;
   Sched sched;
-  float* part_o;             // [2W][n_h][d_c]
+  void* part_o;              // [2W][n_h][d_c], type of the path: a split segment's latent sum over
+                             // its keys, normalised by its own l (so bf16 keeps it as well as obar)
   float* part_ml;            // [2W][2][n_h][2]: (m, l) per latent-column half (ml_index)
   void* obar;                // [R][n_h][d_c] (type of the path)
   int* err;
@@ -164,10 +165,11 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
         for (int r = 0; r < MAX_CPT; ++r)
           if (r < cpt && oj + r * TPH < a.d_c) out[oj + r * TPH] = from_f32<T>(o[r] * inv);
       } else {
-        float* po = a.part_o + ((long long)g.slot * a.n_h + h) * a.d_c;
+        T* po = static_cast<T*>(a.part_o) + ((long long)g.slot * a.n_h + h) * a.d_c;
+        const float inv = 1.f / l;
 #pragma unroll
         for (int r = 0; r < MAX_CPT; ++r)
-          if (r < cpt && oj + r * TPH < a.d_c) po[oj + r * TPH] = o[r];
+          if (r < cpt && oj + r * TPH < a.d_c) po[oj + r * TPH] = from_f32<T>(o[r] * inv);
         if (oj == 0) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -186,13 +188,21 @@ inline size_t smem_bytes(int HG, int d_cr) {
 }  // namespace attn_simt
 
 // ------------------------------------------------------------ combine -----
-// Merges the partial slots of each split row block (log-sum-exp in base 2):
-//   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  obar = sum_s 2^(m_s - m) O_s / l.
+// Merges the partial slots of each split row block (log-sum-exp in base 2);
+// slot s holds its normalised sum N_s = O_s / l_s and (m_s, l_s):
+//   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  obar = sum_s 2^(m_s - m) l_s N_s / l.
 // Block = (split row block, 8 heads), one warp per head.  Lane k gathers the
 // (slot, m, l) of segments k, k + 32, ...; the warp reduces them with
 // shuffles, then each lane accumulates four consecutive latent columns of
 // each 128-column chunk (d_c <= 512) with 16-byte loads.  Slots are added in
 // segment order, so the result is deterministic.
+__device__ __forceinline__ float4 load4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = __ldcg(reinterpret_cast<const uint2*>(p));
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
 __device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
   *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
 }
@@ -203,6 +213,8 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float
 
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial slots come from the attention kernel
   const Sched& S = a.sched;
   const int idx = blockIdx.x;
   if (idx >= S.split_rbs[0]) return;
@@ -244,20 +256,22 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
     float wgt0 = 0.f, wgt1 = 0.f;
     if (sb + lane < s1) {
       slot = S.segs[sb + lane].slot;
-      wgt0 = exp2f(a.part_ml[ml_index(slot, 0, a.n_h, h)] - m[0]);
-      wgt1 = exp2f(a.part_ml[ml_index(slot, 1, a.n_h, h)] - m[1]);
+      const float* ml0 = a.part_ml + ml_index(slot, 0, a.n_h, h);
+      const float* ml1 = a.part_ml + ml_index(slot, 1, a.n_h, h);
+      wgt0 = exp2f(ml0[0] - m[0]) * ml0[1];
+      wgt1 = exp2f(ml1[0] - m[1]) * ml1[1];
     }
     const int cnt = min(32, s1 - sb);
     for (int k = 0; k < cnt; ++k) {
       const int sl = __shfl_sync(0xffffffffu, slot, k);
       const float w0 = __shfl_sync(0xffffffffu, wgt0, k);
       const float w1 = __shfl_sync(0xffffffffu, wgt1, k);
-      const float* src = a.part_o + ((long long)sl * a.n_h + h) * a.d_c;
+      const T* src = static_cast<const T*>(a.part_o) + ((long long)sl * a.n_h + h) * a.d_c;
       float4 v[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int j = c * 128 + 4 * lane;
-        v[c] = j < a.d_c ? __ldcg(reinterpret_cast<const float4*>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[c] = j < a.d_c ? load4(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {

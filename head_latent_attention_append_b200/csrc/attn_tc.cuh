@@ -214,6 +214,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap rmap16,
                    const __grid_constant__ CUtensorMap rmap32, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_trigger();
+  pdl_wait();  // the schedule and Q_abs come from earlier kernels
   if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
     if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
     return;
@@ -728,33 +730,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const float lrow = ls[r] + ls[128 + r];
           if (!(ok = pair_sync())) break;
           // A whole row block is normalised into obar (bf16); a piece of a
-          // split row block leaves its unnormalised sum and this CTA's (m, l)
-          // in its slot.
+          // split row block is normalised by its own sum into its partial
+          // slot (bf16) and leaves this CTA's (m, l) beside it.
           const bool whole = g.slot < 0;
           const float inv = 1.f / lrow;
+          __nv_bfloat16* const dst_row =
+              whole ? static_cast<__nv_bfloat16*>(a.obar) + ((long long)g.rb * a.n_h + r) * a.d_c
+                    : static_cast<__nv_bfloat16*>(a.part_o) + ((long long)g.slot * a.n_h + r) * a.d_c;
           for (int cc = hc0; cc < hc1; ++cc) {
             uint32_t v[32];
             tmem_ld32(tO + cc * 32, v);
             tmem_ld_wait();
             if (r < a.n_h) {
-              const int col = (int)rank * dh + cc * 32;
-              if (whole) {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.obar) +
-                                                      ((long long)g.rb * a.n_h + r) * a.d_c + col);
-                float dummy = 0.f;
+              uint4* dst = reinterpret_cast<uint4*>(dst_row + (int)rank * dh + cc * 32);
+              float dummy = 0.f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  uint4 o;
-                  o.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv, dummy);
-                  o.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv, dummy);
-                  o.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv, dummy);
-                  o.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv, dummy);
-                  dst[q] = o;
-                }
-              } else {
-                uint4* dst = reinterpret_cast<uint4*>(a.part_o + ((long long)g.slot * a.n_h + r) * a.d_c + col);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              for (int q = 0; q < 4; ++q) {
+                uint4 o;
+                o.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv, dummy);
+                o.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv, dummy);
+                o.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv, dummy);
+                o.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv, dummy);
+                dst[q] = o;
               }
             }
           }

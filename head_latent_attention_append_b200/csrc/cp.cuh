@@ -109,13 +109,6 @@ __global__ void __launch_bounds__(1024) cp_sched_kernel(SchedArgs a, CpWindow wi
     }
 }
 
-__device__ __forceinline__ float4 load4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-  const uint2 u = __ldcg(reinterpret_cast<const uint2*>(p));
-  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
-}
 
 // Per (row block, head): merges the row block's segment slots into the
 // normalised latent sum obar_r (type T) and lse_r = m + log2 l.  A row block
@@ -163,9 +156,11 @@ __global__ void __launch_bounds__(256) cp_combine_kernel(AttnArgs a, T* obar_out
   for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = s0; s < s1; ++s) {
     const int slot = S.segs[s].slot;
-    const float w0 = exp2f(a.part_ml[ml_index(slot, 0, a.n_h, h)] - m[0]);
-    const float w1 = exp2f(a.part_ml[ml_index(slot, 1, a.n_h, h)] - m[1]);
-    const float* src = a.part_o + ((long long)slot * a.n_h + h) * a.d_c;
+    const float* ml0 = a.part_ml + ml_index(slot, 0, a.n_h, h);
+    const float* ml1 = a.part_ml + ml_index(slot, 1, a.n_h, h);
+    const float w0 = exp2f(ml0[0] - m[0]) * ml0[1];  // the slots hold normalised sums
+    const float w1 = exp2f(ml1[0] - m[1]) * ml1[1];
+    const T* src = static_cast<const T*>(a.part_o) + ((long long)slot * a.n_h + h) * a.d_c;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int j = c * 128 + 4 * lane;

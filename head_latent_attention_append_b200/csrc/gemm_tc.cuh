@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the activations (and the split-K scratch) come from the previous kernel
 
   if (warp == 0) {
     // TMA producer: runs ahead across items as far as the ring allows.
@@ -246,6 +248,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 constexpr int MAX_SPLITS = 32;
 template <int BN, class Epi>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const Args g, const Epi epi) {
+  pdl_trigger();
+  pdl_wait();
   const int bz = blockIdx.z, slices = BN / 8;
   const int tile_m = blockIdx.x >> 1, half = blockIdx.x & 1;
   const int tile_n = blockIdx.y / slices, slice = blockIdx.y % slices;

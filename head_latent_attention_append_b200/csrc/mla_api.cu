@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 
 #include <cudaTypedefs.h>
 
@@ -113,6 +114,33 @@ int cache_row(const mla_dims& d) { return d.d_c + (d.rope_key_per_head ? d.n_h :
 // (shared memory: 32 keys plus up to 16 heads' queries, fp32).
 constexpr int kSimtMaxRow = 1024;
 
+// A second stream of the library's own for work that depends only on the
+// call's inputs and can run beside the main chain (the attention schedule,
+// which needs only the lengths, runs beside the query projections).  One
+// non-blocking stream and two timing-free events per host thread and device,
+// created on first use and kept until the thread exits.  The fork/join
+// through the events is ordinary stream ordering, so it also holds inside a
+// CUDA graph capture of the caller's stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+cudaError_t side_stream(SideStream** out) {
+  static thread_local SideStream table[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  SideStream& t = table[dev];
+  if (!t.s) {
+    if ((e = cudaStreamCreateWithFlags(&t.s, cudaStreamNonBlocking))) return e;
+    if ((e = cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming))) return e;
+    if ((e = cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming))) return e;
+  }
+  *out = &t;
+  return cudaSuccess;
+}
+
 mla_status check_dims(const mla_dims* d) {
   if (!d) return MLA_ERR_INVALID_ARG;
   if (d->rope_key_per_head != 0 && d->rope_key_per_head != 1) return MLA_ERR_INVALID_ARG;
@@ -186,7 +214,7 @@ Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false) {
     P.segs = o;       o = align_up(o + sizeof(Seg) * (size_t)(W + R), 256);
     P.rb_first = o;   o = align_up(o + sizeof(int) * (size_t)(R + 1), 256);
     P.split_rbs = o;  o = align_up(o + sizeof(int) * (size_t)(2 * W + 1), 256);
-    P.part_o = o;     o = align_up(o + sizeof(float) * slots * d.n_h * d.d_c, 256);
+    P.part_o = o;     o = align_up(o + e * slots * d.n_h * d.d_c, 256);
     P.part_ml = o;    o = align_up(o + sizeof(float) * slots * 2 * d.n_h * 2, 256);
     P.obar = o;       o = align_up(o + e * (size_t)R * d.n_h * d.d_c, 256);
   }
@@ -200,6 +228,26 @@ T* at(void* base, size_t off) {
 }
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// Launches `kernel` with programmatic stream serialization: it may begin
+// while the previous kernel in the stream is finishing, and waits for it
+// (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda at build time).
@@ -300,12 +348,12 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   if (e != cudaSuccess) return e;
   ++g_launches;
   const int items = tiles * splits;
-  kfn<<<dim3(std::min(items, sms)), gemm_tc::THREADS, smem, st>>>(mapW, mapX, g, epi);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pdl(kfn, dim3(std::min(items, sms)), dim3(gemm_tc::THREADS), smem, st, mapW, mapX, g, epi)))
+    return e;
   if (splits > 1) {
     ++g_launches;
-    gemm_tc::splitk_reduce_kernel<BN, Epi><<<dim3(2 * tm, tn * (BN / 8), batch), 256, 0, st>>>(g, epi);
-    e = cudaGetLastError();
+    e = launch_pdl(gemm_tc::splitk_reduce_kernel<BN, Epi>, dim3(2 * tm, tn * (BN / 8), batch), dim3(256), 0, st,
+                   g, epi);
   }
   return e;
 }
@@ -407,6 +455,56 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   const int din = d_in(d);
   int* err = at<int>(ws, P.hdr);
   cudaError_t e;
+  // (0) the attention schedule, on the side stream: it depends only on the
+  // lengths, so it runs while the query projections below stream weights
+  // (one 512-thread CTA, small enough to sit on an SM beside a GEMM CTA).
+  SideStream* side = nullptr;
+  if ((e = side_stream(&side))) return cuda_status(e);
+  Sched S{at<int>(ws, P.tile_start), at<int>(ws, P.worker_seg), at<Seg>(ws, P.segs), at<int>(ws, P.rb_first),
+          at<int>(ws, P.split_rbs)};
+  AttnArgs aa{};
+  aa.qabs = at<T>(ws, P.qabs);
+  aa.qrows = P.qrows;
+  aa.cache = cache;
+  aa.page_table = page_table;
+  aa.max_pages = max_pages;
+  aa.num_pages = num_pages;
+  aa.page_size = d.page_size;
+  aa.n_h = d.n_h; aa.d_c = d.d_c; aa.d_r = d.d_r; aa.d_cr = d_cr;
+  aa.q_row = q_row;
+  aa.rope_per_head = d.rope_key_per_head;
+  aa.kv_len = kv_len; aa.uniform_kv_len = uniform_kv_len; aa.n_q = n_q; aa.max_kv_len = max_kv_len;
+  aa.sched = S;
+  aa.part_o = at<T>(ws, P.part_o);
+  aa.part_ml = at<float>(ws, P.part_ml);
+  aa.obar = at<T>(ws, P.obar);
+  aa.err = err;
+
+  // bf16 with one shared RoPE key runs on the tensor cores; per-head RoPE
+  // keys (whose position term is a per-head contraction, not one dense
+  // product over the shared row) and fp32 run on the CUDA cores.
+  const bool kTensorCores = sizeof(T) == 2 && !d.rope_key_per_head;
+  // fp32: heads per CTA a power of two so that 256 threads split evenly.
+  int HG = 16;
+  while (HG > d.n_h) HG >>= 1;
+  const int G = kTensorCores ? 2 : ceil_div(d.n_h, HG);
+  // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
+  int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
+                       : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
+  {
+    SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
+    ++g_launches;
+    if ((e = cudaEventRecord(side->fork, st)) || (e = cudaStreamWaitEvent(side->s, side->fork, 0)))
+      return cuda_status(e);
+    if (cp) {
+      cp_sched_kernel<<<1, 512, 0, side->s>>>(sa, cp->win);
+    } else {
+      const size_t sched_smem = R + 1 <= kSchedSmemRb ? sizeof(int) * (size_t)(R + 1) : 0;
+      if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
+      sched_kernel<<<1, 512, sched_smem, side->s>>>(sa);
+    }
+    if ((e = cudaGetLastError()) || (e = cudaEventRecord(side->join, side->s))) return cuda_status(e);
+  }
   // (1) query latent.
   const void* src = hq;
   if (d.d_cq > 0) {
@@ -437,50 +535,8 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
                      R, d.d_c, d.d_h, d.n_h, epi, ws, P, st)))
       return cuda_status(e);
   }
-  // (4) schedule.
-  Sched S{at<int>(ws, P.tile_start), at<int>(ws, P.worker_seg), at<Seg>(ws, P.segs), at<int>(ws, P.rb_first),
-          at<int>(ws, P.split_rbs)};
-  AttnArgs aa{};
-  aa.qabs = at<T>(ws, P.qabs);
-  aa.qrows = P.qrows;
-  aa.cache = cache;
-  aa.page_table = page_table;
-  aa.max_pages = max_pages;
-  aa.num_pages = num_pages;
-  aa.page_size = d.page_size;
-  aa.n_h = d.n_h; aa.d_c = d.d_c; aa.d_r = d.d_r; aa.d_cr = d_cr;
-  aa.q_row = q_row;
-  aa.rope_per_head = d.rope_key_per_head;
-  aa.kv_len = kv_len; aa.uniform_kv_len = uniform_kv_len; aa.n_q = n_q; aa.max_kv_len = max_kv_len;
-  aa.sched = S;
-  aa.part_o = at<float>(ws, P.part_o);
-  aa.part_ml = at<float>(ws, P.part_ml);
-  aa.obar = at<T>(ws, P.obar);
-  aa.err = err;
-
-  // bf16 with one shared RoPE key runs on the tensor cores; per-head RoPE
-  // keys (whose position term is a per-head contraction, not one dense
-  // product over the shared row) and fp32 run on the CUDA cores.
-  const bool kTensorCores = sizeof(T) == 2 && !d.rope_key_per_head;
-  // fp32: heads per CTA a power of two so that 256 threads split evenly.
-  int HG = 16;
-  while (HG > d.n_h) HG >>= 1;
-  const int G = kTensorCores ? 2 : ceil_div(d.n_h, HG);
-  // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
-  int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
-                       : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
-  {
-    SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
-    ++g_launches;
-    if (cp) {
-      cp_sched_kernel<<<1, 1024, 0, st>>>(sa, cp->win);
-    } else {
-      const size_t sched_smem = R + 1 <= kSchedSmemRb ? sizeof(int) * (size_t)(R + 1) : 0;
-      if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
-      sched_kernel<<<1, 1024, sched_smem, st>>>(sa);
-    }
-    if ((e = cudaGetLastError())) return cuda_status(e);
-  }
+  // The schedule has run on the side stream beside steps (1) - (3).
+  if ((e = cudaStreamWaitEvent(st, side->join, 0))) return cuda_status(e);
   // (5) attention on the latent cache, (6) combine of split row blocks.
   if (kTensorCores) {
     CUtensorMap map;
@@ -494,7 +550,9 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     if ((e = set_smem_once(attn_tc::attn_tc_kernel, attn_tc::SMEM_BYTES))) return cuda_status(e);
     ++g_launches;
     prof_mark(st, true);
-    attn_tc::attn_tc_kernel<<<dim3(2 * W), attn_tc::THREADS, attn_tc::SMEM_BYTES, st>>>(map, rmap16, rmap32, pp);
+    if ((e = launch_pdl(attn_tc::attn_tc_kernel, dim3(2 * W), dim3(attn_tc::THREADS), attn_tc::SMEM_BYTES, st, map,
+                        rmap16, rmap32, pp)))
+      return cuda_status(e);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
   } else {
@@ -515,7 +573,8 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   }
   {
     ++g_launches;
-    combine_kernel<T><<<dim3(2 * W, ceil_div(d.n_h, 8)), 256, 0, st>>>(aa);
+    if ((e = launch_pdl(combine_kernel<T>, dim3(2 * W, ceil_div(d.n_h, 8)), dim3(256), 0, st, aa)))
+      return cuda_status(e);
     if ((e = cudaGetLastError())) return cuda_status(e);
   }
   // (7) o_h = W_UV,h obar_h.

@@ -103,6 +103,17 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __all_sync(0xffffffffu, ok);
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel of its stream is finishing.  pdl_wait() blocks until
+// that kernel has completed and its memory operations are visible: every
+// kernel calls it before its first global-memory access, so only prologue
+// work (barrier init, TMEM allocation, descriptor prefetch) overlaps.  In a
+// kernel launched without the attribute it returns at once.
+// pdl_trigger() lets the next kernel in the stream begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
