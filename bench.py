@@ -378,6 +378,19 @@ def l2_plan(unique_bytes: int, l2_bytes: int):
                f"{l2_bytes / 1e6:.0f} MB L2)")
 
 
+def with_batch(name: str, batch: int) -> str:
+    """Registers (once) and returns a copy of workload `name` with `batch`
+    sequences, for profiling the same kernels on a smaller case."""
+    import dataclasses
+    from head_latent_attention_append_b200 import synth
+    if batch <= 0 or batch == synth.WORKLOADS[name].B:
+        return name
+    key = f"{name}_b{batch}"
+    if key not in synth.WORKLOADS:
+        synth.WORKLOADS[key] = dataclasses.replace(synth.WORKLOADS[name], name=key, B=batch)
+    return key
+
+
 def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
     """Every figure of one workload: the device-timed step (median of repeated
     regions of `steps` graph replays), the attention kernel's own time and its
@@ -580,7 +593,7 @@ def run_ours(args):
     ws, rank, local = dist_setup()
     peaks = load_peaks()
     want_cpu = rank == 0 and ws == 1 and not args.no_cpu_baseline
-    head = measure_workload(args.workload, args, ws, local, peaks, want_cpu)
+    head = measure_workload(with_batch(args.workload, args.batch), args, ws, local, peaks, want_cpu)
     line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic"}
@@ -609,6 +622,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="report only the headline workload (no prefill / ragged objects)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run the workload with this many sequences instead of its own B (smaller profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

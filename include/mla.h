@@ -24,9 +24,16 @@
  *     before anything is launched.  Errors found on the device (a page id out
  *     of range, a length out of range) are OR-ed into an error word at the
  *     start of the caller's workspace and never trap; mla_get_error reads it.
- *   - The library allocates no device memory.  Scratch space is the caller's
- *     `workspace`, sized by the *_workspace_bytes queries; the workspace of a
- *     call must not be used by another call that may run at the same time.
+ *   - The library calls no device-memory allocator.  Scratch space is the
+ *     caller's `workspace`, sized by the *_workspace_bytes queries; the
+ *     workspace of a call must not be used by another call that may run at
+ *     the same time.  (The workspace-free append keeps a fixed ~2 MiB array in
+ *     the library's own device memory instead, see below.)  Decode creates,
+ *     on its first call in a host thread on a device, one non-blocking CUDA
+ *     stream and two events of its own: the attention schedule runs there
+ *     beside the query projections, forked from and joined back into
+ *     `stream` (which a CUDA graph capture of `stream` records as ordinary
+ *     dependencies); make that first call before any stream capture.
  *   - Cache layout: [num_pages, page_size, d_cr]; row (page p, slot s) holds
  *     [c_t (d_c) | k_R,t (d_r)] (d_cr = d_c + d_r; with per-head RoPE keys
  *     d_cr = d_c + n_h*d_r, see mla_dims) for the token whose position is
