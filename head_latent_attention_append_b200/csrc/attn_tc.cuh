@@ -1,10 +1,10 @@
 // Absorbed latent attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA),
-// one 2-CTA cluster per worker.
+// one 2-CTA cluster per worker, the two CTAs working as one MMA pair.
 //
 // What it computes is the same as attn_simt.cuh ("ai-decoupled-rope-mla",
-// absorbed score and output equations): for one query token, all of its heads
-// form the M = 128 rows (heads beyond n_h are zero rows), and for each 64-key
-// cache page
+// absorbed score and output equations): for one query token, its heads form
+// the M = 128 rows (heads beyond n_h are zero rows), and for each 64-key cache
+// page
 //   S  = Q_abs [128 x d_cr] * page^T [d_cr x 64]      (content + position
 //        score in one contraction: the cache row is [c | k_R] and the query
 //        row is [q~ | q_R], both pre-scaled by s*log2(e))
@@ -14,60 +14,54 @@
 // Attention Meets RoPE": one shared position key; the latent is shared by
 // construction).
 //
-// B200 layout.  TMEM (128 lanes x 512 fp32 columns per SM) cannot hold the
-// 128 x 512 fp32 latent accumulator of one token next to anything else, so
-// the two CTAs of a cluster split the columns of the cache row:
-//   rank 0: latent columns [0, d_c/2) and the first ra RoPE-key columns
-//   rank 1: latent columns [d_c/2, d_c) and the other rb = d_r - ra,
-// with ra = 16 * (d_r / 32) so that both score shares are whole 16-column MMA
-// steps and, for d_r = 32 or 64, equal.  Each CTA streams only its own
-// columns of every page (no byte is read twice from HBM) and computes the
-// partial score over them into TMEM.  The partial goes to the peer as fp16
-// (saturated at +-65504, log2 units) through distributed shared memory; each
-// CTA's softmax threads add the peer's partial to their own exact fp32 one.
-// So the two CTAs' scores differ by the rounding of one fp16 partial and each
-// runs its own softmax state (m, l) for its half of the latent columns: each
-// half is normalised by its own state, and split row blocks leave one
-// (m, l) per half.  fp16's 11-bit significand keeps this well below the
-// rounding the bf16 cache rows put into every score (a bf16 exchange doubled
-// the error against the fp64 oracle once logits reach ~30).
+// B200 layout.  The 128 x d_c fp32 accumulator of one token fills a whole
+// SM's TMEM, so the work is spread over a CTA pair with cta_group::2 MMAs:
+// each CTA owns 64 of the heads (64 rows of A) and keeps the complete score
+// and softmax state for them, and half of B's columns come from each CTA:
+//   score:  B = the page rows; CTA r supplies keys [32r, 32r + 32) of all
+//           d_cr columns, and holds S for its heads over all 64 keys;
+//   output: B = the page's latent columns; CTA r supplies columns
+//           [r d_c/2, (r + 1) d_c/2) of all 64 keys, and holds O for its heads
+//           over all d_c columns (lanes 0-63: the first half, 64-127: the
+//           second, d_c/2 TMEM columns).
+// No partial score crosses between the CTAs and each CTA's softmax covers
+// only its own 64 heads.  The RoPE key is read as one more 64-column chunk of
+// the row (columns past d_cr read as zero; the query's RoPE part is padded
+// with zeros to match).
 //
-// TMEM columns: O [0, d_c/2), two score buffers S0 [256, 320) and
-// S1 [320, 384), the latent part of this CTA's Q slice from 384 (at most 128
-// columns).  A score buffer is free again as soon as the sender and the
-// finishers have read it (the peer's partial is not waited for first), so the
-// DSMEM latency of the exchange stays out of the score pipeline.
+// TMEM columns: O [0, d_c/2), two score buffers S0 [256, 288) and
+// S1 [288, 320) (64 keys of 64 heads: 32 columns each), the first (up to six)
+// 64-column chunks of the CTA's Q rows from 320 (an A operand in TMEM holds
+// the CTA's rows twice, 32 columns per chunk).  The rest of Q (at most three
+// chunks) sits in shared memory.
 //
 // Shared memory (1024-byte aligned pieces):
-//   three 16 KB exchange buffers, filled by the peer with bulk copies (one
-//     4 KB copy per sender warp per page) that complete on this CTA's
-//     mbarrier; each goes back to the peer with a tcgen05.commit multicast
-//     onto the peer's credit barrier after the page's P*V, which is issued
-//     only once the finishers have read the buffer (a remote arrive from the
-//     finishers themselves is a cluster-scope release that stalls the warp);
-//   a 16 KB staging block for this CTA's outgoing partial;
-//   score ring, 2 slots: this CTA's columns of a page (its latent chunks and
-//     its RoPE share, loaded with a 16- or 32-column box swizzled to 32 or 64
-//     bytes), freed as soon as the page's score MMA completes;
-//   latent ring, 2 slots: the page's latent columns again (4 chunks) for
-//     P*V, freed by P*V.  The second read is an L2 hit (the first was a few
-//     microseconds earlier), so HBM still sees every byte once;
-//   the RoPE part of the Q slice (SS MMA operand, swizzled like the page's
-//     RoPE share) and the 16 KB P tile (SS P*V operand);
-//   two 1 KB slots of half-row maxima for the finishers' pair exchange
-//     (a segment's row sums borrow the idle one).
-// Segment metadata and page ids are loaded a step ahead so no global load
-// sits on a page's critical path.
+//   score ring, 3 slots: the CTA's 32 keys of every 64-column chunk of a page
+//     (128-byte swizzled, 4 KB per chunk), freed when the page's score MMA
+//     completes;
+//   latent ring, 2 slots: all 64 keys of the CTA's d_c/128 latent chunks
+//     (8 KB each), freed by P*V.  The page went through L2 for the score
+//     ring a few microseconds earlier, so HBM sees its bytes once;
+//   the shared-memory part of Q, two P tiles (64 heads x 64 keys bf16, the
+//   A operand of P*V), a staging tile through which the TMEM part of Q
+//   passes (loaded coalesced, read back one row per thread), and the
+//   row-max / row-sum exchange slots.
+// The page loads of both CTAs complete on the even CTA's barriers (the MMA
+// issuer's).  The last page of a row block, whose tail rows may hold
+// anything (NaN included), lands on a barrier of the CTA's own instead, so
+// that its softmax threads can clear those rows before P*V multiplies them
+// by zero.
 //
-// Warp roles (512 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
-// allocator and latent-ring TMA producer, warp 1 = score-MMA issuer, warp 3 =
-// P*V-MMA issuer (all warp-uniform; one elected lane issues), warps 4-7 =
-// sender (reads each page's own partial score from TMEM, ships it to the
-// peer, loads each segment's Q slice), warps 8-11 and 12-15 = the two
-// finisher halves (keys 0-31 and 32-63 of every row: score, softmax, P, and
-// half of O in the epilogue); thread r of any of these owns row r = TMEM
-// lane r.  Two score buffers let the score MMA of page t+1 run while the
-// finishers work on page t.  Every wait is bounded (sm100::mbar_wait).
+// Warp roles (384 threads): warp 0 = score-ring TMA producer, warp 2 = TMEM
+// allocator and latent-ring producer, warp 1 of the even CTA = MMA issuer
+// (order: S(t), then P*V(t-1), so each page's softmax overlaps the next
+// page's score MMA), warps 4-11 = softmax.  Softmax thread (lane quarter q,
+// column half c) owns TMEM lane L = 32q + lane: head L mod 64, keys
+// [32 (L div 64) + 16c, +16) of each page, and O columns
+// [(L div 64) d_c/2 + c d_c/4, +d_c/4); the four threads of a head agree on
+// its row max through shared memory and a 128-thread named barrier, and each
+// keeps a partial row sum (the same rescalings), added at the end.  Every
+// wait is bounded (sm100::mbar_wait).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
@@ -76,49 +70,41 @@ namespace mla {
 namespace attn_tc {
 using namespace sm100;
 
-constexpr int THREADS = 512;
-constexpr int KT = 64;                        // keys per tile (one page)
-constexpr int CHUNK_BYTES = 64 * 64 * 2;      // 64 keys x 64 bf16 columns
-constexpr int MAX_PV = 4;                     // latent chunks per CTA per page (d_c <= 512)
-constexpr int MAX_ROPE = 32;                  // RoPE-key columns per CTA (d_r <= 64)
-constexpr int SGROUPS = 2;                    // score ring: a page's own columns, freed by its score MMA
-constexpr int VGROUPS = 2;                    // latent ring: the page's latent columns again, freed by P*V
-constexpr int XBUF = 3;                       // exchange buffers per CTA (credit-controlled)
-constexpr int ROPE_OFF = MAX_PV * CHUNK_BYTES;  // a score slot: latent chunks, then the RoPE share
-constexpr int SG_BYTES = ROPE_OFF + KT * MAX_ROPE * 2;
-constexpr int VG_BYTES = MAX_PV * CHUNK_BYTES;
-constexpr int X_BYTES = 128 * KT * 2;         // one fp16 partial-score tile
-constexpr int QR_BYTES = 128 * MAX_ROPE * 2;  // the RoPE part of the Q slice
-constexpr int P_BYTES = 128 * KT * 2;         // P tile: 128 rows x 64 keys bf16
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384, TM_COLS = 512;
+constexpr int THREADS = 384;
+constexpr int KT = 64;                    // keys per page
+constexpr int HEADS = 64;                 // query rows per CTA
+constexpr int CH_S = 32 * 128;            // 32 keys x 64 bf16 columns (4 KB)
+constexpr int CH_V = KT * 128;            // 64 keys x 64 bf16 columns (8 KB)
+constexpr int MAX_NK = 9;                 // 64-column chunks of a cache row (d_c <= 512, d_r <= 64)
+constexpr int MAX_NPV = 4;                // latent chunks per CTA (d_c / 128)
+constexpr int MAX_TS = 6;                 // chunks of Q held in TMEM
+constexpr int SGS = 3, VGS = 2;           // ring slots
+constexpr int SG_BYTES = MAX_NK * CH_S;   // 36 KB
+constexpr int VG_BYTES = MAX_NPV * CH_V;  // 32 KB
+constexpr int QS_BYTES = 3 * CH_V;        // the chunks of Q beyond the first MAX_TS (64 rows each)
+constexpr int P_BYTES = HEADS * KT * 2;   // 8 KB
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320, TM_COLS = 512;
 
-// The exchange buffers and the credit barriers sit at the same offsets in
-// both CTAs (the peer addresses them through mapa).
-constexpr int OFF_X = 0;
-constexpr int OFF_XS = OFF_X + XBUF * X_BYTES;    // outgoing partial, staged for the bulk copy
-constexpr int OFF_SG = OFF_XS + X_BYTES;
-constexpr int OFF_VG = OFF_SG + SGROUPS * SG_BYTES;
-constexpr int OFF_QR = OFF_VG + VGROUPS * VG_BYTES;
-constexpr int OFF_P = OFF_QR + QR_BYTES;
-constexpr int OFF_MH = OFF_P + P_BYTES;           // half-row maxima [2][2][128] fp32 (sums reuse a slot)
-constexpr int OFF_BAR = OFF_MH + 2 * 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * XBUF + 2 * SGROUPS + 2 * VGROUPS + 2 + 2 + 1 + 1 + 3 + 4;
+constexpr int OFF_SG = 0;
+constexpr int OFF_VG = OFF_SG + SGS * SG_BYTES;
+constexpr int OFF_QS = OFF_VG + VGS * VG_BYTES;
+constexpr int OFF_P = OFF_QS + QS_BYTES;
+constexpr int OFF_STG = OFF_P + 2 * P_BYTES;       // staging tile for the TMEM part of Q (64 rows x 128 B)
+constexpr int OFF_MX = OFF_STG + CH_V;             // [2][64] float4: the four partial maxima of a head
+constexpr int OFF_LS = OFF_MX + 2 * HEADS * 16;    // [64] float4: the four partial sums
+constexpr int OFF_BAR = OFF_LS + HEADS * 16;
+constexpr int NUM_BARS = 2 * SGS + 3 * VGS + 2 + 2 + 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-static_assert(OFF_SG % 1024 == 0 && OFF_VG % 1024 == 0 && OFF_QR % 1024 == 0 && OFF_P % 1024 == 0 &&
-                  SG_BYTES % 1024 == 0,
+static_assert(OFF_VG % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0 && OFF_STG % 1024 == 0 &&
+                  SG_BYTES % 1024 == 0 &&
+                  VG_BYTES % 1024 == 0,
               "swizzled operands need 1024-byte aligned tiles");
 // No slack for aligning the base: the kernel has no static shared memory, so
 // its dynamic block starts on a 1024-byte boundary (the kernel checks this
 // and reports MLA_ERR_UNSUPPORTED otherwise).
 constexpr size_t SMEM_BYTES = SMEM_USED;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA can have");
-
-struct Params {
-  AttnArgs a;
-  int npv;     // latent chunks per CTA (d_c / 128)
-  int ra, rb;  // RoPE-key columns scored by rank 0 and rank 1 (multiples of 16, ra + rb = d_r)
-};
 
 // 2^x with the MUFU ex2 instruction (flush-to-zero; ~2 ulp), used for the
 // softmax weights, which are rounded to bf16 right after.
@@ -128,13 +114,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b, float& sum) {
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  sum += __low2float(v) + __high2float(v);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// ------------------------------------------------------- cluster helpers
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -149,632 +133,578 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
-// a peer CTA's, completing as transaction bytes on the peer's mbarrier
-// `bar_cluster_addr`.  One copy carries what would otherwise be many small
-// remote stores, each with its own transaction-count update at the peer.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster_addr, uint32_t src_smem, uint32_t bytes,
-                                                  uint32_t bar_cluster_addr) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst_cluster_addr),
-      "r"(src_smem), "r"(bytes), "r"(bar_cluster_addr)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until the sources of this thread's committed bulk copies have been read.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Arrives once on the mbarrier at the same shared-memory offset in every CTA
-// of `cta_mask` when every tcgen05 operation this thread issued has completed.
-__device__ __forceinline__ void tc_commit_to(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"(cta_mask)
-      : "memory");
-}
 // Asks L2 to fetch `bytes` (a multiple of 16) from global memory ahead of use.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
-// Partial scores travel between the CTAs as fp16 pairs, saturated at
-// +-65504 (one conversion per pair).
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  uint32_t u;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
-  return u;
-}
-// Exact fp16 pair -> two floats with integer work and one multiply per value
-// (no conversion-pipe work): the 15 bits below a half's sign, moved to an
-// fp32's exponent and significand positions, are its value times 2^-112
-// (subnormal halves included, as fp32 subnormals); the sign moves over.
-__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
-  const float lo = __uint_as_float((u << 13) & 0x0fffe000u) * 0x1p112f;
-  const float hi = __uint_as_float((u >> 3) & 0x0fffe000u) * 0x1p112f;
-  return make_float2(__uint_as_float(__float_as_uint(lo) | ((u << 16) & 0x80000000u)),
-                     __uint_as_float(__float_as_uint(hi) | (u & 0x80000000u)));
-}
+// A shared-memory descriptor advanced by `bytes` (its address field counts
+// 16-byte units; every operand here stays below 256 KB, so no carry leaves it).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 
-// Byte offset, in an exchange tile and in the P tile, of 16-byte piece u
-// (0..7) of row r's 64 16-bit values: row r at r * 128, piece u at
-// (u ^ (r & 7)) * 16.  This is the 128-byte-swizzled K-major operand layout
-// (8-row groups of 1 KB) the P*V MMA reads P in; each warp's 32 rows are one
-// contiguous 4 KB block (one bulk copy), and the eight rows a quarter-warp
-// touches at once fall in eight bank groups.
-constexpr int X_WARP_BYTES = 32 * KT * 2;
-__device__ __forceinline__ uint32_t x_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
-// Byte offset of 16-byte piece u of row r in the RoPE part of the Q slice,
-// rows of rw * 2 bytes swizzled to that width (64-byte rows: piece ^ row
-// bits 1-2; 32-byte rows: piece ^ row bit 2), matching sdesc_swz.
-__device__ __forceinline__ uint32_t qr_off(int r, int u, int rw) {
-  return rw == 32 ? (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) : (uint32_t)(r * 32 + ((u ^ ((r >> 2) & 1)) << 4));
-}
+// Walks a worker's segments page by page: (segment, tile) and the cache page
+// id, with the next page's id loaded one step ahead.
+struct PageWalk {
+  const Seg* segs;
+  const int32_t* page_table;
+  int max_pages, n_q;
+  int si, seg_hi, t;
+  Seg g, gn;
+  bool more;
+  int page_next;
+  __device__ void start(int seg_lo) {
+    si = seg_lo;
+    more = si < seg_hi;
+    if (!more) return;
+    g = segs[si];
+    gn = si + 1 < seg_hi ? segs[si + 1] : g;
+    t = g.t_lo;
+    page_next = page_table[(long long)(g.rb / n_q) * max_pages + t];
+  }
+  // The current page's id; steps to the next page.
+  __device__ int next(Seg& cur, int& tile) {
+    cur = g;
+    tile = t;
+    const int page = page_next;
+    if (++t >= g.t_hi) {
+      if (++si < seg_hi) {
+        g = gn;
+        if (si + 1 < seg_hi) gn = segs[si + 1];
+        t = g.t_lo;
+      } else {
+        more = false;
+      }
+    }
+    if (more) page_next = page_table[(long long)(g.rb / n_q) * max_pages + t];
+    return page;
+  }
+};
 
+template <int NPV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap rmap16,
-                   const __grid_constant__ CUtensorMap rmap32, const Params p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapV,
+                   const AttnArgs a) {
+  constexpr int NCH = 2 * NPV;                       // latent chunks of a row
+  constexpr int NK = NCH + 1;                        // + the RoPE chunk
+  constexpr int NTS = NK < MAX_TS ? NK : MAX_TS;     // chunks of Q in TMEM
+  constexpr int NSS = NK - NTS;                      // chunks of Q in shared memory
+  static_assert(NPV >= 1 && NPV <= MAX_NPV && NSS * CH_V <= QS_BYTES, "latent width");
   extern __shared__ __align__(1024) uint8_t smem[];
   pdl_trigger();
-  pdl_wait();  // the schedule and Q_abs come from earlier kernels
   if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
-    if (threadIdx.x == 0) flag_error(p.a.err, kErrLayout);
+    if (threadIdx.x == 0) flag_error(a.err, kErrLayout);
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* x_full = bars;               // [XBUF] the peer's partial has landed here
-  uint64_t* x_free = x_full + XBUF;      // [XBUF] the peer has consumed what this CTA sent
-  uint64_t* sg_full = x_free + XBUF;     // [SGROUPS]
-  uint64_t* sg_empty = sg_full + SGROUPS;
-  uint64_t* vg_full = sg_empty + SGROUPS;  // [VGROUPS]
-  uint64_t* vg_empty = vg_full + VGROUPS;
-  uint64_t* s_full = vg_empty + VGROUPS;   // [2] own partial score in buffer b
-  uint64_t* s_free = s_full + 2;           // [2] the sender and the finishers have read buffer b
-  uint64_t* p_ready = s_free + 2;          // P of the current page is in the P tile
-  uint64_t* pv_done = p_ready + 1;         // P*V of the current page has completed
-  uint64_t* q_ready = pv_done + 1;
-  uint64_t* o_free = q_ready + 1;
-  uint64_t* final_bar = q_ready + 2;
-  uint64_t* pair_bars = q_ready + 3;       // [4]: the two finisher warps of a lane quarter
+  uint64_t* sg_full = bars;                // [SGS] both CTAs' score chunks landed (even CTA's)
+  uint64_t* sg_empty = sg_full + SGS;      // [SGS] the page's score MMA is done (both CTAs)
+  uint64_t* vg_full = sg_empty + SGS;      // [VGS] both CTAs' latent chunks landed (even CTA's)
+  uint64_t* vg_empty = vg_full + VGS;      // [VGS] the page's P*V is done (both CTAs)
+  uint64_t* vg_part = vg_empty + VGS;      // [VGS] this CTA's chunks of a row block's last page landed
+  uint64_t* s_full = vg_part + VGS;        // [2] S of the page in buffer b is complete (both CTAs)
+  uint64_t* p_ready = s_full + 2;          // [2] both CTAs' P of the page are in their P tiles (even CTA's)
+  uint64_t* pv_done = p_ready + 2;         // [2] P*V of the page has completed (both CTAs)
+  uint64_t* q_ready = pv_done + 2;         // a segment's Q rows are in place in both CTAs (even CTA's)
+  uint64_t* o_free = q_ready + 1;          // both CTAs have read a segment's O (even CTA's)
+  uint64_t* final_bar = o_free + 1;        // the MMA issuer's last commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
   const int w = blockIdx.x >> 1;
-  const AttnArgs& a = p.a;
-  const int npv = p.npv, dh = npv * 64;
-  const int c_lo = (int)rank * npv;                // first latent chunk of this CTA
-  const int rw = rank ? p.rb : p.ra;               // RoPE-key columns this CTA scores (0, 16 or 32)
-  const int rx = a.d_c + (rank ? p.ra : 0);        // and the first of them
-  const CUtensorMap* rmap = rw == 32 ? &rmap32 : &rmap16;
-  const uint64_t rswz = rw == 32 ? kSwizzle64 : kSwizzle32;
-  const Seg* segs = a.sched.segs;
-  const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
   if (tid == 32) {
-    for (int i = 0; i < XBUF; ++i) {
-      mbar_init(&x_full[i], 1);  // own expect_tx + the peer's bytes
-      mbar_init(&x_free[i], 1);  // the peer's P*V commit
+    for (int i = 0; i < SGS; ++i) {
+      mbar_init(&sg_full[i], 1);   // the even CTA's arrive.expect_tx + both CTAs' bytes
+      mbar_init(&sg_empty[i], 1);  // commit of the score MMA
     }
-    for (int i = 0; i < SGROUPS; ++i) {
-      mbar_init(&sg_full[i], 1);
-      mbar_init(&sg_empty[i], 1);
-    }
-    for (int i = 0; i < VGROUPS; ++i) {
+    for (int i = 0; i < VGS; ++i) {
       mbar_init(&vg_full[i], 1);
       mbar_init(&vg_empty[i], 1);
+      mbar_init(&vg_part[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 384);  // sender + finishers
+      mbar_init(&p_ready[i], 16);  // one arrive per softmax warp of both CTAs
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_ready, 256);  // finishers
-    mbar_init(pv_done, 1);
-    mbar_init(q_ready, 128);  // sender
-    mbar_init(o_free, 256);   // finishers
-    mbar_init(final_bar, 2);  // one commit per issuer warp
-    for (int i = 0; i < 4; ++i) mbar_init(&pair_bars[i], 64);
+    mbar_init(q_ready, 16);
+    mbar_init(o_free, 16);
+    mbar_init(final_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, TM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, TM_COLS);
+    tmem_relinquish_pair();
   }
   if (tid == 0) {
-    tma_prefetch_desc(&tmap);
-    if (rw) tma_prefetch_desc(rmap);
+    tma_prefetch_desc(&mapS);
+    tma_prefetch_desc(&mapV);
   }
   __syncthreads();
-  cluster_sync_all();  // the peer's barriers exist before anyone signals them
+  cluster_sync_all();  // the peer's barriers and TMEM exist before anyone signals them
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // Everything above overlaps the previous kernel's tail; the schedule and
+  // Q_abs come from earlier kernels.
+  pdl_wait();
+  const Seg* segs = a.sched.segs;
+  const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 
   if (warp == 0 || warp == 2) {
     // ---------------------------------------------------- TMA producers
-    // Warp 0 fills the score ring with this CTA's columns of each page;
-    // warp 2 fills the latent ring with the page's latent columns again
-    // (an L2 hit: the score ring read them a few microseconds earlier).
-    // Metadata loads run one step ahead: the next segment while this one
-    // streams, the next page id while this page waits for its ring slot.
+    // Warp 0 fills the score ring (this CTA's 32 keys of every chunk), warp
+    // 2 the latent ring (all 64 keys of this CTA's latent chunks); both
+    // complete on the even CTA's barriers, except a row block's last page in
+    // the latent ring (see above).
     const bool score_ring = warp == 0;
-    const int nring = score_ring ? SGROUPS : VGROUPS;
-    const int ring_bytes = score_ring ? SG_BYTES : VG_BYTES;
-    const int rope_cols = score_ring ? rw : 0;
-    uint8_t* ring = smem + (score_ring ? OFF_SG : OFF_VG);
+    const int nslots = score_ring ? SGS : VGS;
     uint64_t* full = score_ring ? sg_full : vg_full;
     uint64_t* empty = score_ring ? sg_empty : vg_empty;
-    uint32_t cnt = 0;
-    if (seg_lo < seg_hi) {
-      int si = seg_lo;
-      Seg g = segs[si];
-      Seg gn = si + 1 < seg_hi ? segs[si + 1] : g;
-      int t = g.t_lo;
-      int page_n = a.page_table[(long long)(g.rb / a.n_q) * a.max_pages + t];
-      bool more = true;
-      while (more) {
-        int page = page_n;
-        if (++t >= g.t_hi) {
-          if (++si < seg_hi) {
-            g = gn;
-            if (si + 1 < seg_hi) gn = segs[si + 1];
-            t = g.t_lo;
-          } else {
-            more = false;
-          }
-        }
-        if (more) page_n = a.page_table[(long long)(g.rb / a.n_q) * a.max_pages + t];
-        const uint32_t gs = cnt % nring;
-        if (!mbar_wait_warp(&empty[gs], ((cnt / nring) & 1) ^ 1, abort_flag, a.err)) break;
-        if (page < 0 || page >= a.num_pages) {
-          if (rank == 0 && score_ring && elect_one()) flag_error(a.err, kErrBounds);
-          page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
-        }
-        if (elect_one()) {
-          mbar_arrive_expect_tx(&full[gs], npv * CHUNK_BYTES + rope_cols * KT * 2);
-          for (int q = 0; q < npv; ++q)
-            tma_load_2d(ring + gs * ring_bytes + q * CHUNK_BYTES, &tmap, (c_lo + q) * 64, page * KT, &full[gs]);
-          if (rope_cols) tma_load_2d(ring + gs * ring_bytes + ROPE_OFF, rmap, rx, page * KT, &full[gs]);
-        }
-        __syncwarp();
-        ++cnt;
+    uint8_t* ring = smem + (score_ring ? OFF_SG : OFF_VG);
+    const int slot_bytes = score_ring ? SG_BYTES : VG_BYTES;
+    const uint32_t full_even = map_peer(smem_u32(full), 0);
+    PageWalk pw{segs, a.page_table, a.max_pages, a.n_q, 0, seg_hi, 0, Seg{}, Seg{}, false, 0};
+    pw.start(seg_lo);
+    static_assert(VGS == 2, "two latent slots");
+    uint32_t cnt = 0, part_cnt0 = 0, part_cnt1 = 0;  // tail loads per latent slot
+    while (pw.more) {
+      Seg g;
+      int t;
+      int page = pw.next(g, t);
+      const uint32_t s = cnt % nslots;
+      if (!mbar_wait_warp(&empty[s], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err)) break;
+      if (page < 0 || page >= a.num_pages) {
+        if (rank == 0 && score_ring && elect_one()) flag_error(a.err, kErrBounds);
+        page = 0;  // keep the pipeline's byte counts; outputs are flagged invalid
       }
+      const bool tail = (t + 1) * KT > g.nkeys;  // keys past the row block's end in this page
+      uint8_t* dst = ring + s * slot_bytes;
+      if (elect_one()) {
+        if (score_ring) {
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * NK * CH_S);
+          for (int c = 0; c < NK; ++c)
+            tma_load_2d_pair(dst + c * CH_S, &mapS, 64 * c, page * KT + (int)rank * 32, full_even + 8 * s);
+        } else if (!tail) {
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * NPV * CH_V);
+          for (int q = 0; q < NPV; ++q)
+            tma_load_2d_pair(dst + q * CH_V, &mapV, ((int)rank * NPV + q) * 64, page * KT, full_even + 8 * s);
+        } else {
+          mbar_arrive_expect_tx(&vg_part[s], NPV * CH_V);
+          for (int q = 0; q < NPV; ++q)
+            tma_load_2d(dst + q * CH_V, &mapV, ((int)rank * NPV + q) * 64, page * KT, &vg_part[s]);
+          if (rank == 0) mbar_arrive(&full[s]);  // the phase still advances; p_ready covers the bytes
+        }
+      }
+      __syncwarp();
+      if (!score_ring && tail) {
+        if (s == 0) ++part_cnt0;
+        else ++part_cnt1;
+      }
+      ++cnt;
     }
     if (*abort_flag) {
-      // Let every copy already issued land before the CTA can exit.
-      for (uint32_t q = 0; q < (uint32_t)nring && q < cnt; ++q) {
-        const uint32_t last = q + nring * ((cnt - 1 - q) / nring);
-        mbar_wait_warp(&full[q], (last / nring) & 1, abort_flag, nullptr, 50000000ull, false);
-      }
+      // Let every copy already issued land before the CTA can exit (the even
+      // CTA's barriers count the odd CTA's bytes too).
+      if (rank == 0)
+        for (uint32_t q = 0; q < (uint32_t)nslots && q < cnt; ++q) {
+          const uint32_t last = q + nslots * ((cnt - 1 - q) / nslots);
+          mbar_wait_warp(&full[q], (last / nslots) & 1, abort_flag, nullptr, 50000000ull, false);
+        }
+      if (!score_ring)
+        for (int q = 0; q < VGS; ++q) {
+          const uint32_t n_q = q == 0 ? part_cnt0 : part_cnt1;
+          if (n_q) mbar_wait_warp(&vg_part[q], (n_q - 1) & 1, abort_flag, nullptr, 50000000ull, false);
+        }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------- score-MMA issuer
-    // Page t's partial score goes into buffer t & 1, free once the sender and
-    // the finishers have read page t - 2's scores from it.
-    const uint32_t tS = tbase + TM_S, tQ = tbase + TM_Q;
-    const uint32_t sSG = smem_u32(smem + OFF_SG), sQR = smem_u32(smem + OFF_QR);
+  } else if (warp == 1 && rank == 0) {
+    // ------------------------------------------------------- MMA issuer
+    const uint32_t tS = tbase + TM_S, tO = tbase + TM_O, tQ = tbase + TM_Q;
+    const uint64_t dS0 = sdesc_sw128(smem_u32(smem + OFF_SG), 16, 1024);
+    const uint64_t dQ0 = sdesc_sw128(smem_u32(smem + OFF_QS), 16, 1024);
+    const uint64_t dP0 = sdesc_sw128(smem_u32(smem + OFF_P), 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(smem_u32(smem + OFF_VG), CH_V, 1024);  // MN-major: LBO = chunk stride
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);
-    uint32_t tg = 0, seg_k = 0;
+    const uint32_t idV2 = idesc_bf16(128, 256, 0, 1), idV1 = idesc_bf16(128, 128, 0, 1);
     bool ok = true;
-    Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const Seg g = gn;
-      if (si + 1 < seg_hi) gn = segs[si + 1];  // in flight while this segment runs
-      const int n = g.t_hi - g.t_lo;
-      if (!(ok = mbar_wait_warp(q_ready, seg_k & 1, abort_flag, a.err))) break;
+    // P*V of page pj: waits for both CTAs' P (and, at a segment's first page,
+    // for both CTAs to have read the previous segment's O).
+    auto issue_pv = [&](uint32_t pj, bool first, uint32_t sk) -> bool {
+      const uint32_t vs = pj % VGS;
+      bool r_ok = mbar_wait(&vg_full[vs], (pj / VGS) & 1, abort_flag, a.err);
+      if (r_ok && first && sk > 0) r_ok = mbar_wait(o_free, (sk - 1) & 1, abort_flag, a.err);
+      if (r_ok) r_ok = mbar_wait(&p_ready[pj & 1], (pj >> 1) & 1, abort_flag, a.err);
+      if (!__all_sync(0xffffffffu, r_ok)) return false;
       tc_fence_after();
-      for (int i = 0; i < n; ++i, ++tg) {
-        const uint32_t b = tg & 1;
-        if (tg >= 2 && !(ok = mbar_wait_warp(&s_free[b], ((tg - 2) >> 1) & 1, abort_flag, a.err))) break;
-        const uint32_t gs = tg % SGROUPS;
-        if (!(ok = mbar_wait_warp(&sg_full[gs], (tg / SGROUPS) & 1, abort_flag, a.err))) break;
-        tc_fence_after();
-        if (elect_one()) {
-          const uint32_t gb = sSG + gs * SG_BYTES, d = tS + b * KT;
-          for (int q = 0; q < npv; ++q) {
+      if (elect_one()) {
+        const uint64_t a0 = desc_add(dP0, (pj & 1) * P_BYTES);
+        const uint64_t b0 = desc_add(dV0, vs * VG_BYTES);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_ts(d, tQ + q * 32 + k * 8, sdesc_sw128(gb + q * CHUNK_BYTES + k * 32, 16, 1024), idS,
-                     (q | k) ? 1u : 0u);
-          }
-          // The RoPE share: rows of rw * 2 bytes, swizzled to that width, both
-          // operands in shared memory.
-          for (int k = 0; k < rw / 16; ++k)
-            mma_ss(d, sdesc_swz(sQR + k * 32, 8 * rw * 2, rswz), sdesc_swz(gb + ROPE_OFF + k * 32, 8 * rw * 2, rswz),
-                   idS, 1u);
-          tc_commit(&s_full[b]);
-          tc_commit(&sg_empty[gs]);  // the score ring slot is free once its MMAs are done
+        for (int k = 0; k < KT / 16; ++k) {
+#pragma unroll
+          for (int m = 0; m < (NPV + 1) / 2; ++m)
+            mma_pair_ss(tO + m * 128, desc_add(a0, k * 32), desc_add(b0, m * 2 * CH_V + k * 2048),
+                        (2 * m + 1 < NPV) ? idV2 : idV1, (first && k == 0) ? 0u : 1u);
         }
-        __syncwarp();
+        tc_commit_pair(&pv_done[pj & 1], 3);
+        tc_commit_pair(&vg_empty[vs], 3);
       }
-      ++seg_k;
-    }
-    if (elect_one()) tc_commit(final_bar);
-    __syncwarp();
-    mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
-  } else if (warp == 3) {
-    // ------------------------------------------------------ P*V issuer
-    const uint32_t tO = tbase + TM_O;
-    const uint32_t sVG = smem_u32(smem + OFF_VG), sP = smem_u32(smem + OFF_P);
-    const uint32_t idPV = idesc_bf16(128, dh, 0, 1);
-    uint32_t tg = 0, seg_k = 0;
-    bool ok = true;
-    Seg gn = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-    for (int si = seg_lo; si < seg_hi && ok; ++si) {
-      const Seg g = gn;
-      if (si + 1 < seg_hi) gn = segs[si + 1];
+      __syncwarp();
+      return true;
+    };
+    uint32_t j = 0, seg_k = 0, prev_j = 0, prev_sk = 0;
+    bool have_prev = false, prev_first = false;
+    for (int si = seg_lo; si < seg_hi && ok; ++si, ++seg_k) {
+      const Seg g = segs[si];
       const int n = g.t_hi - g.t_lo;
-      for (int i = 0; i < n; ++i, ++tg) {
-        if (!(ok = mbar_wait_warp(p_ready, tg & 1, abort_flag, a.err))) break;
-        if (i == 0 && seg_k > 0 && !(ok = mbar_wait_warp(o_free, (seg_k - 1) & 1, abort_flag, a.err))) break;
-        const uint32_t vs = tg % VGROUPS;
-        if (!(ok = mbar_wait_warp(&vg_full[vs], (tg / VGROUPS) & 1, abort_flag, a.err))) break;
+      for (int i = 0; i < n; ++i, ++j) {
+        if (i == 0) {
+          // The previous segment's last P*V first, then this segment's Q.
+          if (have_prev && !(ok = issue_pv(prev_j, prev_first, prev_sk))) break;
+          have_prev = false;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_ready, seg_k & 1, abort_flag, a.err)))) break;
+        }
+        const uint32_t gs = j % SGS;
+        if (!(ok = mbar_wait_warp(&sg_full[gs], (j / SGS) & 1, abort_flag, a.err))) break;
         tc_fence_after();
         if (elect_one()) {
+          const uint32_t d = tS + (j & 1) * 32;
+          const uint64_t b0 = desc_add(dS0, gs * SG_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < KT / 16; ++kk)
-            mma_ss(tO, sdesc_sw128(sP + kk * 32, 16, 1024),
-                   sdesc_sw128(sVG + vs * VG_BYTES + kk * 2048, CHUNK_BYTES, 1024), idPV,
-                   (i == 0 && kk == 0) ? 0u : 1u);
-          tc_commit(pv_done);
-          tc_commit(&vg_empty[vs]);
-          // The finishers read exchange buffer tg % XBUF before P_tg was
-          // ready: hand it back to the peer's sender.
-          tc_commit_to(&x_free[tg % XBUF], (uint16_t)(1u << peer));
+          for (int c = 0; c < NK; ++c) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t b = desc_add(b0, c * CH_S + k * 32);
+              if (c < NTS)
+                mma_pair_ts(d, tQ + c * 32 + k * 8, b, idS, (c | k) ? 1u : 0u);
+              else
+                mma_pair_ss(d, desc_add(dQ0, (c - NTS) * CH_V + k * 32), b, idS, (c | k) ? 1u : 0u);
+            }
+          }
+          tc_commit_pair(&s_full[j & 1], 3);
+          tc_commit_pair(&sg_empty[gs], 3);
         }
         __syncwarp();
+        if (have_prev && !(ok = issue_pv(prev_j, prev_first, prev_sk))) break;
+        have_prev = true;
+        prev_j = j;
+        prev_first = i == 0;
+        prev_sk = seg_k;
       }
-      ++seg_k;
     }
-    if (elect_one()) tc_commit(final_bar);
+    if (ok && have_prev) issue_pv(prev_j, prev_first, prev_sk);
+    if (elect_one()) tc_commit_pair(final_bar, 1);
     __syncwarp();
     mbar_wait_warp(final_bar, 0, abort_flag, nullptr, 50000000ull, false);
   } else if (warp >= 4) {
-    // ------------------------------------------- sender and finisher warpgroups
-    // Thread r of either warpgroup owns row r (= TMEM lane r) of the page.
-    const bool sender = warp < 8;
-    const int h = warp >= 12 ? 1 : 0;  // finisher half: keys [32h, 32h + 32)
-    const int r = tid - (sender ? 128 : 256 + 128 * h);
-    const int lane = tid & 31;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    // ---------------------------------------------------------- softmax
+    const int q4 = warp & 3, ch = (warp - 4) >> 2, grp = warp & 1;
+    const int L = q4 * 32 + lane, hl = L & 63, kh = L >> 6, part = kh * 2 + ch;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tbase + lane_off + TM_S, tO = tbase + lane_off + TM_O, tQ = tbase + lane_off + TM_Q;
+    const int head = (int)rank * HEADS + hl;
+    const bool live = head < a.n_h;
+    float* mx = reinterpret_cast<float*>(smem + OFF_MX);  // [2][64][4]
+    float* lsum = reinterpret_cast<float*>(smem + OFF_LS);  // [64][4]
+    const uint32_t p_ready_even = map_peer(smem_u32(p_ready), 0);
+    const uint32_t q_ready_even = map_peer(smem_u32(q_ready), 0);
+    const uint32_t o_free_even = map_peer(smem_u32(o_free), 0);
+    const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
+    // A failed wait clears `ok` (warp-uniform) and the rest of the work is
+    // skipped, but every thread still walks every page and every Q load so
+    // that the named barriers always see all of their threads.
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       bool r_ok = mbar_wait(bar, parity, abort_flag, a.err);
       return __all_sync(0xffffffffu, r_ok);
     };
-
-    if (sender) {
-      // Reads each page's own partial score (all 64 keys of its row) from
-      // TMEM, packs it to fp16, stages it and ships it to the peer with one
-      // bulk copy per warp; also loads each segment's Q slice.
-      uint8_t* sQR = smem + OFF_QR;
-      uint8_t* sXS = smem + OFF_XS;
-      const uint32_t peer_x = map_peer(smem_u32(smem + OFF_X), peer);
-      const uint32_t peer_xbar = map_peer(smem_u32(&x_full[0]), peer);
-      const __nv_bfloat16* qabs = static_cast<const __nv_bfloat16*>(a.qabs);
-      // Row r of this CTA's Q slice: the latent chunks c_lo .. c_lo + npv - 1
-      // into TMEM, the RoPE share into shared memory.
-      auto load_q = [&](int rb) {
-        const uint4* src =
-            (r < a.n_h) ? reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + r) * a.d_cr) : nullptr;
-        for (int q = 0; q < npv; ++q) {
-          uint32_t wv[32];
+    auto signal_even = [&](uint32_t bar_even) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(bar_even);
+    };
+    // This CTA's Q rows of row block rb: chunks [0, NTS) into TMEM (lane L
+    // holds head hl; both lane halves take the row), the rest into shared
+    // memory (one thread per row and chunk).
+    // A segment's Q rows: q_issue() issues every global load into registers
+    // before any store (coalesced: softmax thread tau = 0..255 takes 16-byte
+    // pieces tau and tau + 256 of each 64-row x 128-byte chunk, eight threads
+    // per row segment); q_store() writes them.  The next segment's rows are
+    // loaded once the current segment's last score MMA is complete, from L2
+    // (prefetched a few pages earlier).
+    uint4 pv[NK][2];
+    auto q_issue = [&](int rb) {
+      const int tau = tid - 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            uint4 v = src ? __ldg(src + ((c_lo + q) * 64 + u * 8) / 8) : make_uint4(0, 0, 0, 0);
-            wv[4 * u + 0] = v.x;
-            wv[4 * u + 1] = v.y;
-            wv[4 * u + 2] = v.z;
-            wv[4 * u + 3] = v.w;
-          }
-          tmem_st32(tQ + q * 32, wv);
+      for (int c = 0; c < NK; ++c)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int pc = tau + 256 * h, r = pc >> 3, e0 = 64 * c + 8 * (pc & 7), hd = (int)rank * HEADS + r;
+          pv[c][h] = (ok && hd < a.n_h && e0 < a.q_row)
+                         ? __ldg(reinterpret_cast<const uint4*>(qabs + ((long long)rb * a.qrows + hd) * a.q_row + e0))
+                         : make_uint4(0, 0, 0, 0);
         }
-        for (int u = 0; u < rw / 8; ++u) {
-          const uint4 v = src ? __ldg(src + (rx + u * 8) / 8) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(sQR + qr_off(r, u, rw)) = v;
+    };
+    auto q_store = [&]() {
+      const int tau = tid - 128;
+      // Chunks [NTS, NK) go straight to their shared-memory tiles.
+#pragma unroll
+      for (int s2 = 0; s2 < NSS; ++s2)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int pc = tau + 256 * h, r = pc >> 3, u = pc & 7;
+          *reinterpret_cast<uint4*>(smem + OFF_QS + s2 * CH_V + r * 128 + ((u ^ (r & 7)) << 4)) = pv[NTS + s2][h];
         }
+      // Chunks [0, NTS) pass through the staging tile, one at a time: thread
+      // (L, ch) then stores columns [16 ch, 16 ch + 16) of the chunk for
+      // TMEM lane L (both lane halves hold row L mod 64).
+#pragma unroll
+      for (int c = 0; c < NTS; ++c) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int pc = tau + 256 * h, r = pc >> 3, u = pc & 7;
+          *reinterpret_cast<uint4*>(smem + OFF_STG + r * 128 + ((u ^ (r & 7)) << 4)) = pv[c][h];
+        }
+        named_bar_sync(3, 256);
+        uint32_t wv[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = *reinterpret_cast<const uint4*>(smem + OFF_STG + hl * 128 + (((4 * ch + v) ^ (hl & 7)) << 4));
+          wv[4 * v + 0] = x.x;
+          wv[4 * v + 1] = x.y;
+          wv[4 * v + 2] = x.z;
+          wv[4 * v + 3] = x.w;
+        }
+        if (ok) tmem_st16(tQ + 32 * c + 16 * ch, wv);
+        named_bar_sync(3, 256);
+      }
+      if (ok) {
         fence_proxy_async_smem();  // the MMA (async proxy) reads what the threads wrote
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(q_ready);
-      };
-      // Segment metadata stays in registers, the next segment's loaded a
-      // segment ahead.
-      Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-      Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : Seg{};
-      if (seg_lo < seg_hi) load_q(g_cur.rb);
-      // The next segment's query rows are pulled into L2 while this segment
-      // streams, so loading them at the segment boundary reads L2, not HBM.
-      const uint32_t q_half = (uint32_t)((a.n_h + 1) / 2) * a.d_cr * 2;
-      auto prefetch_q = [&](int rb) {
-        if (tid == 128) {
-          const uint8_t* base = reinterpret_cast<const uint8_t*>(qabs + (long long)rb * a.qrows * a.d_cr);
-          const uint32_t lo = rank ? q_half : 0, hi = rank ? (uint32_t)a.n_h * a.d_cr * 2 : q_half;
-          if (hi > lo) prefetch_l2(base + lo, hi - lo);
-        }
-      };
-      uint32_t tg = 0;
-      for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const Seg g = g_cur;
-        const int n = g.t_hi - g.t_lo;
-        if (si + 1 < seg_hi) prefetch_q(g_nxt.rb);
-        for (int i = 0; i < n; ++i, ++tg) {
-          const uint32_t b = tg & 1, xb = tg % XBUF;
-          if (!(ok = wait_all(&s_full[b], (tg >> 1) & 1))) break;
-          tc_fence_after();
-          uint32_t cur[32];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld32(tS + b * KT + 32 * half, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              cur[16 * half + j] = pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          }
-          // Keys past the row block's end (the tail of its last page) may hold
-          // anything, NaN included; the peer's exchange MMA multiplies every
-          // key of a row by the identity's zeros too, so they travel as 0.
-          const int valid_all = min(KT, g.nkeys - (g.t_lo + i) * KT);
-          if (valid_all < KT) {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) {
-              if (2 * x >= valid_all) cur[x] = 0u;
-              else if (2 * x + 1 >= valid_all) cur[x] &= 0x0000ffffu;
-            }
-          }
-          tc_fence_before();
-          mbar_arrive(&s_free[b]);
-          // The segment's scores are all read after its last page, so the next
-          // segment's Q may replace this one's.
-          if (i + 1 == n && si + 1 < seg_hi) load_q(g_nxt.rb);
-          // The staging block is reused once the copy engine has read it.
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(sXS + x_off(r, u)) =
-                make_uint4(cur[4 * u], cur[4 * u + 1], cur[4 * u + 2], cur[4 * u + 3]);
-          fence_proxy_async_smem();  // the copy engine reads what the threads wrote
-          // The peer's partial of this page will land in exchange buffer xb.
-          if (r == 0) mbar_arrive_expect_tx(&x_full[xb], X_BYTES);
-          // Buffer xb of the peer is free once its finishers have read page
-          // tg - XBUF from it.
-          if (tg >= XBUF && !(ok = wait_all(&x_free[xb], ((tg / XBUF) - 1) & 1))) break;
-          __syncwarp();
-          if (lane == 0) {
-            const uint32_t blk = (uint32_t)((warp & 3) * X_WARP_BYTES);
-            bulk_copy_to_peer(peer_x + xb * X_BYTES + blk, smem_u32(sXS) + blk, X_WARP_BYTES, peer_xbar + xb * 8);
-            bulk_commit();
-          }
-        }
-        g_cur = g_nxt;
-        if (si + 2 < seg_hi) g_nxt = segs[si + 2];
+        signal_even(q_ready_even);
       }
-      // Every credit the peer returns lands before this CTA may exit: wait for
-      // its consumption of the last pages shipped (page p is the (p / XBUF)-th
-      // use of buffer p % XBUF).
-      if (ok)
-        for (uint32_t pg = tg > (uint32_t)XBUF ? tg - XBUF : 0; pg < tg; ++pg)
-          if (!wait_all(&x_free[pg % XBUF], (pg / XBUF) & 1)) break;
-      if (lane == 0) bulk_wait_read_all();  // no copy may still read the staging block at exit
-    } else {
-      // Two finisher warpgroups: half h owns keys [32h, 32h + 32) of every
-      // row and half of O's columns; the two threads of a row (their warps
-      // share a lane quarter) agree on the row max through a bounded
-      // 64-arrival mbarrier.
-      uint64_t* pair_bar = &pair_bars[warp & 3];
-      uint32_t pair_phase = 0;
-      auto pair_sync = [&]() -> bool {
-        mbar_arrive(pair_bar);
-        bool r_ok = mbar_wait(pair_bar, pair_phase & 1, abort_flag, a.err);
-        ++pair_phase;
-        return __all_sync(0xffffffffu, r_ok);
-      };
-      float* mh = reinterpret_cast<float*>(smem + OFF_MH);
-      const int hc0 = h * (dh / 64), hc1 = hc0 + dh / 64;  // this half's 32-column chunks of O
-      Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
-      Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
-      uint8_t* sV = smem + OFF_VG;
-      uint8_t* sPt = smem + OFF_P;
-      const uint8_t* sX = smem + OFF_X;
-      float m_used = -INFINITY, l = 0.f;
-      uint32_t tg = 0;
-      for (int si = seg_lo; si < seg_hi && ok; ++si) {
-        const Seg g = g_cur;
-        const int n = g.t_hi - g.t_lo;
-        for (int i = 0; i < n; ++i, ++tg) {
-          const int t = g.t_lo + i;
-          const uint32_t b = tg & 1;
-          // This CTA's exact partial from TMEM (the buffer is released at
-          // once), then the peer's fp16 partial from the exchange buffer.
-          if (!(ok = wait_all(&s_full[b], (tg >> 1) & 1))) break;
+    };
+    // The next segment's Q rows are pulled into L2 a few pages before they
+    // are loaded (an earlier prefetch would be evicted by the page stream).
+    auto prefetch_q = [&](int rb) {
+      if (tid == 128) {
+        const int h0 = (int)rank * HEADS, h1 = min(a.n_h, h0 + HEADS);
+        if (h1 > h0)
+          prefetch_l2(qabs + ((long long)rb * a.qrows + h0) * a.q_row, (uint32_t)((h1 - h0) * a.q_row * 2));
+      }
+    };
+
+    uint32_t j = 0, part_par = 0;  // bit s: parity of the next tail load in latent slot s
+    Seg g_cur = seg_lo < seg_hi ? segs[seg_lo] : Seg{};
+    Seg g_nxt = seg_lo + 1 < seg_hi ? segs[seg_lo + 1] : g_cur;
+    if (seg_lo < seg_hi) {  // every softmax thread: q_store holds named barriers
+      q_issue(g_cur.rb);
+      q_store();
+    }
+    for (int si = seg_lo; si < seg_hi; ++si) {
+      const Seg g = g_cur;
+      const int n = g.t_hi - g.t_lo;
+      float m_used = -INFINITY, lt = 0.f;
+      for (int i = 0; i < n; ++i, ++j) {
+        const int t = g.t_lo + i;
+        const uint32_t b = j & 1;
+        const int valid_all = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
+        const bool q_next = i + 1 == n && si + 1 < seg_hi;
+        if (si + 1 < seg_hi && i == max(0, n - 6)) prefetch_q(g_nxt.rb);
+        // S of page j is complete, and with it every earlier MMA: P*V of page
+        // j - 2 (issued before S(j)) has released P tile b.
+        ok = ok && wait_all(&s_full[b], (j >> 1) & 1);
+        float s[16];
+        if (ok) {
           tc_fence_after();
-          float s[32];
-          {
-            uint32_t v[32];
-            tmem_ld32(tS + b * KT + 32 * h, v);
-            tmem_ld_wait();
+          uint32_t v[16];
+          tmem_ld16(tS + b * 32 + ch * 16, v);
+          tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
+          for (int x = 0; x < 16; ++x) s[x] = __uint_as_float(v[x]);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) s[x] = 0.f;
+        }
+        const int k0 = kh * 32 + ch * 16;  // this thread's first key of the page
+        if (valid_all < KT) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            if (k0 + x >= valid_all) s[x] = -INFINITY;
+        }
+        float mt;
+        {
+          float m8[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) m8[x] = fmaxf(s[x], s[x + 8]);
+#pragma unroll
+          for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int x = 0; x < w2; ++x) m8[x] = fmaxf(m8[x], m8[x + w2]);
+          mx[(b * HEADS + hl) * 4 + part] = m8[0];
+          named_bar_sync(1 + grp, 128);
+          const float4 m4 = reinterpret_cast<const float4*>(mx)[b * HEADS + hl];
+          mt = fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w));
+        }
+        // Running max with lazy rescaling: O and the sums stay relative to
+        // m_used until a page's max exceeds it by more than 2^8.  The four
+        // threads of a head take the same decision from the same numbers.
+        bool resc = false;
+        float scale = 1.f;
+        if (i == 0) {
+          m_used = mt;
+          lt = 0.f;
+        } else if (mt > m_used + 8.f) {
+          scale = fast_exp2(m_used - mt);
+          m_used = mt;
+          resc = true;
+        }
+        uint32_t pk[8];
+        {
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+          // The row sum adds the fp32 weights (not their bf16 roundings: the
+          // difference is random, 2^-9 relative per key).
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float e0 = fast_exp2(s[2 * u] - m_used), e1 = fast_exp2(s[2 * u + 1] - m_used);
+            ps[u & 3] += e0 + e1;
+            pk[u] = pack_bf16x2(e0, e1);
           }
-          tc_fence_before();
-          mbar_arrive(&s_free[b]);  // the score MMA of page tg + 2 may overwrite it
-          const uint32_t xb = tg % XBUF;
-          if (!(ok = wait_all(&x_full[xb], (tg / XBUF) & 1))) break;
-          {
-            uint4 pv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pv[u] = *reinterpret_cast<const uint4*>(sX + xb * X_BYTES + x_off(r, 4 * h + u));
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint32_t pw[4] = {pv[u].x, pv[u].y, pv[u].z, pv[u].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 y = unpack_f16x2(pw[e]);
-                s[8 * u + 2 * e] += y.x;
-                s[8 * u + 2 * e + 1] += y.y;
-              }
-            }
-          }
-          const int valid_all = min(KT, g.nkeys - t * KT);  // >= 1: every tile holds a key
-          const int valid = valid_all - 32 * h;             // valid keys among this half's 32
-          if (valid < 32) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j >= valid) s[j] = -INFINITY;
-          }
-          float mt;
-          {
-            float mx[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(s[j], s[j + 16]);
-#pragma unroll
-            for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-              for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-            float* slot = mh + (tg & 1) * 256;
-            slot[h * 128 + r] = mx[0];
-            if (!(ok = pair_sync())) break;
-            mt = fmaxf(slot[r], slot[128 + r]);
-          }
-          // Running max with lazy rescaling: O and l stay relative to m_used
-          // until a page's max exceeds it by more than 2^8.  Both halves take
-          // the same decision from the same two numbers.
-          bool resc = false;
-          float scale = 1.f;
-          if (i == 0) {
-            m_used = mt;
-            l = 0.f;
-          } else if (mt > m_used + 8.f) {
-            scale = fast_exp2(m_used - mt);
-            m_used = mt;
-            resc = true;
-          }
-          uint32_t pk[16];
-          float psum;
-          {
-            float ps[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-            // The row sum adds the fp32 weights (not their bf16 roundings: the
-            // difference is random, 2^-9 relative per key, and unpacking the
-            // rounded pairs would cost two more instructions per pair).
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const float e0 = fast_exp2(s[2 * u] - m_used), e1 = fast_exp2(s[2 * u + 1] - m_used);
-              ps[u & 7] += e0 + e1;
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
-              pk[u] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-#pragma unroll
-            for (int w2 = 4; w2 >= 1; w2 >>= 1)
-#pragma unroll
-              for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
-            psum = ps[0];
-          }
-          // The previous page's P*V must be done before P is overwritten or O
-          // rescaled.
-          if (tg > 0) {
-            if (!(ok = wait_all(pv_done, (tg - 1) & 1))) break;
+          lt = lt * scale + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+        }
+        // O is rescaled only after P*V of page j - 1 has completed.
+        if (ok && __any_sync(0xffffffffu, resc)) {
+          ok = wait_all(&pv_done[b ^ 1], ((j - 1) >> 1) & 1);
+          if (ok) {
             tc_fence_after();
-          }
-          if (__any_sync(0xffffffffu, resc)) {
-            for (int cc = hc0; cc < hc1; ++cc) {
+#pragma unroll
+            for (int cc = 0; cc < NPV; ++cc) {
               uint32_t v[32];
-              tmem_ld32(tO + cc * 32, v);
+              tmem_ld32(tO + ch * (NPV * 32) + cc * 32, v);
               tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * scale);
-              tmem_st32(tO + cc * 32, v);
+              for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * scale);
+              tmem_st32(tO + ch * (NPV * 32) + cc * 32, v);
             }
-            l *= scale;
+            tmem_st_wait();
           }
-          // P row r, keys 32h .. 32h + 31: pieces 4h .. 4h + 3 of the
-          // 128-byte-swizzled K-major tile (the SS P*V MMA's A operand).
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(sPt + x_off(r, 4 * h + u)) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          l += psum;
-          if (valid_all < KT) {
-            // Keys past the end: P is 0 there, but 0 * NaN would still poison
-            // O, so clear those rows of this page's latent chunks (once they
-            // have landed).
-            if (!(ok = wait_all(&vg_full[tg % VGROUPS], (tg / VGROUPS) & 1))) break;
-            uint8_t* gb = sV + (tg % VGROUPS) * VG_BYTES;
-            const int rows = KT - valid_all, units = rows * 8 * npv;
-            for (int x = r + 128 * h; x < units; x += 256) {
-              const int q = x / (rows * 8), rem = x - q * rows * 8;
-              *reinterpret_cast<uint4*>(gb + q * CHUNK_BYTES + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
+        }
+        // P row hl, keys k0 .. k0 + 15: 16-byte pieces k0/8 and k0/8 + 1 of
+        // the 128-byte-swizzled K-major tile.
+        if (ok) {
+          uint8_t* prow = smem + OFF_P + b * P_BYTES + hl * 128;
+          const int u0 = k0 >> 3;
+          *reinterpret_cast<uint4*>(prow + ((u0 ^ (hl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ (hl & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        if (ok && (t + 1) * KT > g.nkeys) {
+          // The row block's last page: P is 0 past its end, but 0 * NaN would
+          // still poison O, so clear those rows of this CTA's latent chunks
+          // once they have landed.
+          const uint32_t vs = j % VGS;
+          ok = wait_all(&vg_part[vs], (part_par >> vs) & 1);
+          part_par ^= 1u << vs;
+          if (ok) {
+            uint8_t* vb = smem + OFF_VG + vs * VG_BYTES;
+            const int rows = KT - valid_all, units = rows * 8 * NPV;
+            for (int x = tid - 128; x < units; x += 256) {
+              const int qq = x / (rows * 8), rem = x - qq * rows * 8;
+              *reinterpret_cast<uint4*>(vb + qq * CH_V + (valid_all + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0, 0, 0, 0);
             }
           }
+        }
+        if (ok) {
           fence_proxy_async_smem();  // the MMA (async proxy) reads P and the cleared rows
           tc_fence_before();
-          mbar_arrive(p_ready);
-          if (i + 1 < n) continue;
+          signal_even(p_ready_even + 8 * b);
+        }
+        if (i + 1 < n) continue;
 
-          // ---- epilogue of the segment ----
-          if (!(ok = wait_all(pv_done, tg & 1))) break;
-          tc_fence_after();
-          // Row sum: both halves add the two partial sums in the same order.
-          // The sums borrow the max slot of the previous page: the partner
-          // read that page's maxima before the last pair sync, and the next
-          // page's maxima go there only after the second sync below.
-          float* ls = mh + ((tg + 1) & 1) * 256;
-          ls[h * 128 + r] = l;
-          if (!(ok = pair_sync())) break;
-          const float lrow = ls[r] + ls[128 + r];
-          if (!(ok = pair_sync())) break;
-          // A whole row block is normalised into obar (bf16); a piece of a
-          // split row block is normalised by its own sum into its partial
-          // slot (bf16) and leaves this CTA's (m, l) beside it.
-          const bool whole = g.slot < 0;
-          const float inv = 1.f / lrow;
-          __nv_bfloat16* const dst_row =
-              whole ? static_cast<__nv_bfloat16*>(a.obar) + ((long long)g.rb * a.n_h + r) * a.d_c
-                    : static_cast<__nv_bfloat16*>(a.part_o) + ((long long)g.slot * a.n_h + r) * a.d_c;
-          for (int cc = hc0; cc < hc1; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tO + cc * 32, v);
-            tmem_ld_wait();
-            if (r < a.n_h) {
-              uint4* dst = reinterpret_cast<uint4*>(dst_row + (int)rank * dh + cc * 32);
-              float dummy = 0.f;
+        // ---- end of the segment ----
+        // The next segment's Q replaces this one's (its last score MMA is
+        // complete); then O of this segment, once its last P*V is done.
+        if (q_next) {  // every softmax thread: q_store holds named barriers
+          q_issue(g_nxt.rb);
+          q_store();
+        }
+        ok = ok && wait_all(&pv_done[b], (j >> 1) & 1);
+        lsum[hl * 4 + part] = lt;
+        named_bar_sync(1 + grp, 128);
+        if (ok) tc_fence_after();
+        const float4 l4 = reinterpret_cast<const float4*>(lsum)[hl];
+        const float lrow = (l4.x + l4.y) + (l4.z + l4.w);
+        // A whole row block is normalised into obar (bf16); a piece of a
+        // split row block is normalised by its own sum into its partial slot
+        // and leaves its (m, l) beside it (the same for both column halves).
+        // The rows go out through shared memory (the P tiles and the staging
+        // tile, free now) so that the global stores are coalesced: in round
+        // rho the threads with part == rho write their d_c/4 columns of O,
+        // normalised and rounded, into padded rows, then all softmax threads
+        // store the 64 rows x d_c/4 columns, eight threads per 128 bytes.
+        const bool whole = g.slot < 0;
+        const float inv = 1.f / lrow;
+        constexpr int PPR = 4 * NPV;          // 16-byte pieces per staged row
+        constexpr int SROW = 16 * PPR + 16;   // padded row: consecutive rows start in different banks
+        static_assert(64 * SROW <= 2 * P_BYTES + CH_V, "staged output fits the P and staging tiles");
+        uint8_t* const so = smem + OFF_P;
+        __nv_bfloat16* const obase = whole ? static_cast<__nv_bfloat16*>(a.obar) + (long long)g.rb * a.n_h * a.d_c
+                                           : static_cast<__nv_bfloat16*>(a.part_o) + (long long)g.slot * a.n_h * a.d_c;
+#pragma unroll 1
+        for (int rho = 0; rho < 4; ++rho) {
+          if (ok && part == rho) {
+#pragma unroll
+            for (int cc = 0; cc < NPV; ++cc) {
+              uint32_t v[32];
+              tmem_ld32(tO + ch * (NPV * 32) + cc * 32, v);
+              tmem_ld_wait();
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 uint4 o;
-                o.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv, dummy);
-                o.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv, dummy);
-                o.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv, dummy);
-                o.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv, dummy);
-                dst[q] = o;
+                o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+                o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+                o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+                o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+                *reinterpret_cast<uint4*>(so + hl * SROW + (4 * cc + q) * 16) = o;
               }
             }
           }
-          if (!whole && h == 0 && r < a.n_h) {
-            float* ml = a.part_ml + ml_index(g.slot, (int)rank, a.n_h, r);
+          named_bar_sync(3, 256);
+#pragma unroll
+          for (int m = 0; m < NPV; ++m) {
+            const int pc = (tid - 128) + 256 * m, r = pc / PPR, pp = pc - r * PPR;
+            const int hd = (int)rank * HEADS + r;
+            if (ok && hd < a.n_h)
+              *reinterpret_cast<uint4*>(obase + (long long)hd * a.d_c + rho * (NPV * 32) + 8 * pp) =
+                  *reinterpret_cast<const uint4*>(so + r * SROW + 16 * pp);
+          }
+          named_bar_sync(3, 256);
+        }
+        if (ok && !whole && part == 0 && live) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float* ml = a.part_ml + ml_index(g.slot, half, a.n_h, head);
             ml[0] = m_used;
             ml[1] = lrow;
           }
-          tc_fence_before();
-          mbar_arrive(o_free);
         }
-        g_cur = g_nxt;
-        if (si + 2 < seg_hi) g_nxt = segs[si + 2];
+        if (ok) {
+          tc_fence_before();
+          signal_even(o_free_even);
+        }
       }
+      g_cur = g_nxt;
+      if (si + 2 < seg_hi) g_nxt = segs[si + 2];
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // no CTA leaves while its peer may still write into it
+  cluster_sync_all();  // no CTA leaves while its peer may still use its shared memory or TMEM
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tbase, TM_COLS);
+    tmem_dealloc_pair(tbase, TM_COLS);
   }
 }
 

@@ -249,6 +249,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 
+// The tensor-core attention kernel for a latent width of 128 * NPV.
+template <int NPV>
+cudaError_t launch_attn_tc(const CUtensorMap& mapS, const CUtensorMap& mapV, const AttnArgs& aa, int W,
+                           cudaStream_t st) {
+  auto kfn = attn_tc::attn_tc_kernel<NPV>;
+  cudaError_t e = set_smem_once(kfn, attn_tc::SMEM_BYTES);
+  if (e) return e;
+  return launch_pdl(kfn, dim3(2 * W), dim3(attn_tc::THREADS), attn_tc::SMEM_BYTES, st, mapS, mapV, aa);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda at build time).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -264,24 +274,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2D view of the page pool: rows = num_pages * page_size tokens, columns =
-// d_c + d_r bf16; boxes of 64 tokens x 64 columns, 128-byte swizzle.
-// Columns past d_c + d_r read as zero.
 // The cache as a 2-D tensor [rows = num_pages * 64][d_cr] bf16, read in boxes
-// of `box_cols` columns x 64 rows swizzled to the box's row width (64 columns:
-// 128 bytes; 32: 64 bytes; 16: 32 bytes).
-bool encode_cache_map(CUtensorMap* map, const void* cache, int d_cr, long long rows, int box_cols) {
+// of 64 columns x `box_rows` rows with 128-byte swizzle.  Columns past d_cr
+// read as zero (the RoPE chunk of a row narrower than 64 columns).
+bool encode_cache_map(CUtensorMap* map, const void* cache, int d_cr, long long rows, int box_rows) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)d_cr, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)d_cr * 2};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, 64};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estride[2] = {1, 1};
-  const CUtensorMapSwizzle swz = box_cols == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
-                                 : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(cache), gdim, gstride, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -539,20 +543,21 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   if ((e = cudaStreamWaitEvent(st, side->join, 0))) return cuda_status(e);
   // (5) attention on the latent cache, (6) combine of split row blocks.
   if (kTensorCores) {
-    CUtensorMap map;
+    // Score ring: 32-row boxes (one CTA's keys of a page); latent ring:
+    // 64-row boxes.
+    CUtensorMap mapS, mapV;
     const long long rows = (long long)num_pages * d.page_size;
-    CUtensorMap rmap16, rmap32;
-    if (!encode_cache_map(&map, cache, d_cr, rows, 64) || !encode_cache_map(&rmap16, cache, d_cr, rows, 16) ||
-        !encode_cache_map(&rmap32, cache, d_cr, rows, 32))
+    if (!encode_cache_map(&mapS, cache, d_cr, rows, 32) || !encode_cache_map(&mapV, cache, d_cr, rows, 64))
       return MLA_ERR_CUDA;
-    const int ra = 16 * (d.d_r / 32);  // rank 0's RoPE-key share; rank 1 scores the other d_r - ra
-    attn_tc::Params pp{aa, d.d_c / 128, ra, d.d_r - ra};
-    if ((e = set_smem_once(attn_tc::attn_tc_kernel, attn_tc::SMEM_BYTES))) return cuda_status(e);
     ++g_launches;
     prof_mark(st, true);
-    if ((e = launch_pdl(attn_tc::attn_tc_kernel, dim3(2 * W), dim3(attn_tc::THREADS), attn_tc::SMEM_BYTES, st, map,
-                        rmap16, rmap32, pp)))
-      return cuda_status(e);
+    switch (d.d_c / 128) {
+      case 1: e = launch_attn_tc<1>(mapS, mapV, aa, W, st); break;
+      case 2: e = launch_attn_tc<2>(mapS, mapV, aa, W, st); break;
+      case 3: e = launch_attn_tc<3>(mapS, mapV, aa, W, st); break;
+      default: e = launch_attn_tc<4>(mapS, mapV, aa, W, st); break;
+    }
+    if (e) return cuda_status(e);
     prof_mark(st, false);
     if ((e = cudaGetLastError())) return cuda_status(e);
   } else {

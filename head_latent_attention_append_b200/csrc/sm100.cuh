@@ -180,6 +180,80 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// ------------------------------------------------ CTA-pair (cta_group::2) forms
+// One MMA of a CTA pair computes M = 128 rows split 64 per CTA: each CTA
+// supplies its own 64 rows of A and half of B's N columns (from its own shared
+// memory or TMEM at the same addresses), and holds its 64 x N slice of D as
+// 128 TMEM lanes x N/2 columns: lanes 0-63 carry columns [0, N/2) (the part
+// of B that CTA 0 supplies), lanes 64-127 columns [N/2, N).  An A operand in
+// TMEM holds the CTA's 64 rows twice, in lanes 0-63 and 64-127.  Only the even
+// CTA issues; allocation, commit and deallocation name both.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {  // whole warp, both CTAs
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {  // whole warp, both CTAs
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc] over the CTA pair.
+__device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc] over the CTA pair.
+__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives once on the mbarrier at this shared-memory offset in every CTA of
+// `cta_mask` when the pair MMAs this thread issued have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+// 2D tiled load into this CTA's shared memory whose bytes complete on the
+// mbarrier at cluster address `bar_cluster_addr`, which may be the other
+// CTA's of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cluster_addr) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(bar_cluster_addr)
+      : "memory");
+}
+// Arrive on an mbarrier at a cluster address (this CTA's or the other's of the
+// pair).  Threads that wrote an MMA operand (after fence.proxy.async for
+// shared memory, tcgen05.wait::st for TMEM) or finished reading TMEM (after
+// tcgen05.fence::before_thread_sync) report so to the issuing CTA this way;
+// the default release semantics at CTA scope keep the arrive cheap (a
+// cluster-scope release measured 0.6-1.4 us per arrive here).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32) of this CTA.  It has
+// no time limit, so code that uses it keeps every participating thread
+// arriving the same number of times even after a failed wait.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes
 // with CU_TENSOR_MAP_SWIZZLE_128B for 128-byte rows; the swizzle atom is 8
 // rows x 128 B = 1024 B and must be 1024-byte aligned).
