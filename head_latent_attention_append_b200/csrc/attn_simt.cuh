@@ -194,8 +194,8 @@ inline size_t smem_bytes(int HG, int d_cr) {
 // Block = (split row block, 8 heads), one warp per head.  Lane k gathers the
 // (slot, m, l) of segments k, k + 32, ...; the warp reduces them with
 // shuffles, then each lane accumulates four consecutive latent columns of
-// each 128-column chunk (d_c <= 512) with 16-byte loads.  Slots are added in
-// segment order, so the result is deterministic.
+// each 128-column chunk (d_c <= 512), two slots' loads in flight at a time.
+// Slots are added in segment order, so the result is deterministic.
 __device__ __forceinline__ float4 load4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
   const uint2 u = __ldcg(reinterpret_cast<const uint2*>(p));
@@ -217,70 +217,120 @@ __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial slots come from the attention kernel
   const Sched& S = a.sched;
   const int idx = blockIdx.x;
+  const int W = gridDim.x >> 1;
   if (idx >= S.split_rbs[0]) return;
-  const int rb = S.split_rbs[1 + idx];
+  const int s0 = S.split_rbs[1 + idx];  // the row block's first segment; the others follow it
+  const int nall = S.worker_seg[W];
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (h >= a.n_h) return;
-  const int s0 = S.rb_seg_first[rb], s1 = S.rb_seg_first[rb + 1];
-  // Row max and sum over the segments, for each latent-column half.
-  float m[2] = {-INFINITY, -INFINITY};
-  for (int s = s0 + lane; s < s1; s += 32)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) m[hf] = fmaxf(m[hf], a.part_ml[ml_index(S.segs[s].slot, hf, a.n_h, h)]);
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m[hf] = fmaxf(m[hf], __shfl_xor_sync(0xffffffffu, m[hf], o));
-  float l[2] = {0.f, 0.f};
-  for (int s = s0 + lane; s < s1; s += 32)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const float* ml = a.part_ml + ml_index(S.segs[s].slot, hf, a.n_h, h);
-      l[hf] += exp2f(ml[0] - m[hf]) * ml[1];
-    }
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], o);
-  const float inv[2] = {1.f / l[0], 1.f / l[1]};
+  // Lane k reads segment s0 + k; the row block's segments are the leading
+  // lanes with its row block id.
+  Seg gk;
+  gk.rb = -1;
+  gk.slot = 0;
+  if (s0 + lane < nall) gk = S.segs[s0 + lane];
+  const int rb = __shfl_sync(0xffffffffu, gk.rb, 0);
+  const uint32_t same = __ballot_sync(0xffffffffu, gk.rb == rb);
+  const int lead = __ffs(~same) - 1;  // -1: all 32 lanes belong to rb
+  const int s1 = lead < 0 ? S.rb_seg_first[rb + 1] : s0 + lead;
   const int half_cols = a.d_c / 2;
   T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
-  // All four 128-column chunks (d_c <= 512) at once, so a warp's loads are in
-  // flight together.
   float4 acc[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sb = s0; sb < s1; sb += 32) {
-    // Lane k holds segment sb + k's slot and weights; broadcast in order.
-    int slot = 0;
-    float wgt0 = 0.f, wgt1 = 0.f;
-    if (sb + lane < s1) {
-      slot = S.segs[sb + lane].slot;
-      const float* ml0 = a.part_ml + ml_index(slot, 0, a.n_h, h);
-      const float* ml1 = a.part_ml + ml_index(slot, 1, a.n_h, h);
-      wgt0 = exp2f(ml0[0] - m[0]) * ml0[1];
-      wgt1 = exp2f(ml1[0] - m[1]) * ml1[1];
+  // Adds the rows of slots sa and sb (if has_b) with weights (w0, w1) for
+  // the two column halves; both slots' loads are in flight together.
+  auto add2 = [&](int sa, float wa0, float wa1, bool has_b, int sb, float wb0, float wb1) {
+    const T* pa = static_cast<const T*>(a.part_o) + ((long long)sa * a.n_h + h) * a.d_c;
+    const T* pb = static_cast<const T*>(a.part_o) + ((long long)sb * a.n_h + h) * a.d_c;
+    float4 va[4], vb[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = c * 128 + 4 * lane;
+      va[c] = j < a.d_c ? load4(pa + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[c] = (has_b && j < a.d_c) ? load4(pb + j) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const int cnt = min(32, s1 - sb);
-    for (int k = 0; k < cnt; ++k) {
-      const int sl = __shfl_sync(0xffffffffu, slot, k);
-      const float w0 = __shfl_sync(0xffffffffu, wgt0, k);
-      const float w1 = __shfl_sync(0xffffffffu, wgt1, k);
-      const T* src = static_cast<const T*>(a.part_o) + ((long long)sl * a.n_h + h) * a.d_c;
-      float4 v[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = c * 128 + 4 * lane;
-        v[c] = j < a.d_c ? load4(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int c = 0; c < 4; ++c) {
+      const bool lo = (c * 128 + 4 * lane) < half_cols;
+      const float x = lo ? wa0 : wa1, y = lo ? wb0 : wb1;
+      acc[c].x += x * va[c].x + y * vb[c].x;
+      acc[c].y += x * va[c].y + y * vb[c].y;
+      acc[c].z += x * va[c].z + y * vb[c].z;
+      acc[c].w += x * va[c].w + y * vb[c].w;
+    }
+  };
+  float inv[2] = {1.f, 1.f};
+  if (s1 - s0 <= 32) {
+    // One round trip for the segments (above), one for the (m, l) pairs and
+    // the rows, which do not depend on each other.
+    const int nseg = s1 - s0;
+    const int slot = gk.slot;
+    float mk[2] = {-INFINITY, -INFINITY}, lk[2] = {0.f, 0.f};
+    if (lane < nseg) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float w = (c * 128 + 4 * lane) < half_cols ? w0 : w1;
-        acc[c].x += w * v[c].x;
-        acc[c].y += w * v[c].y;
-        acc[c].z += w * v[c].z;
-        acc[c].w += w * v[c].w;
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + ml_index(slot, hf, a.n_h, h));
+        mk[hf] = ml.x;
+        lk[hf] = ml.y;
       }
+    }
+    float w[2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float m = mk[hf];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      w[hf] = lane < nseg ? exp2f(mk[hf] - m) * lk[hf] : 0.f;
+      float l = w[hf];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      inv[hf] = 1.f / l;
+    }
+    for (int k = 0; k < nseg; k += 2) {
+      const bool has_b = k + 1 < nseg;
+      const int kb = has_b ? k + 1 : k;
+      add2(__shfl_sync(0xffffffffu, slot, k), __shfl_sync(0xffffffffu, w[0], k), __shfl_sync(0xffffffffu, w[1], k),
+           has_b, __shfl_sync(0xffffffffu, slot, kb), __shfl_sync(0xffffffffu, w[0], kb),
+           __shfl_sync(0xffffffffu, w[1], kb));
+    }
+  } else {
+    // More than 32 segments: the same in batches of 32.
+    float m[2] = {-INFINITY, -INFINITY};
+    for (int s = s0 + lane; s < s1; s += 32)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) m[hf] = fmaxf(m[hf], a.part_ml[ml_index(S.segs[s].slot, hf, a.n_h, h)]);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m[hf] = fmaxf(m[hf], __shfl_xor_sync(0xffffffffu, m[hf], o));
+    float l[2] = {0.f, 0.f};
+    for (int sb = s0; sb < s1; sb += 32) {
+      int slot = 0;
+      float w0 = 0.f, w1 = 0.f;
+      if (sb + lane < s1) {
+        slot = S.segs[sb + lane].slot;
+        const float* ml0 = a.part_ml + ml_index(slot, 0, a.n_h, h);
+        const float* ml1 = a.part_ml + ml_index(slot, 1, a.n_h, h);
+        w0 = exp2f(ml0[0] - m[0]) * ml0[1];
+        w1 = exp2f(ml1[0] - m[1]) * ml1[1];
+      }
+      l[0] += w0;
+      l[1] += w1;
+      const int cnt = min(32, s1 - sb);
+      for (int k = 0; k < cnt; k += 2) {
+        const bool has_b = k + 1 < cnt;
+        const int kb = has_b ? k + 1 : k;
+        add2(__shfl_sync(0xffffffffu, slot, k), __shfl_sync(0xffffffffu, w0, k), __shfl_sync(0xffffffffu, w1, k),
+             has_b, __shfl_sync(0xffffffffu, slot, kb), __shfl_sync(0xffffffffu, w0, kb),
+             __shfl_sync(0xffffffffu, w1, kb));
+      }
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], o);
+      inv[hf] = 1.f / l[hf];
     }
   }
 #pragma unroll

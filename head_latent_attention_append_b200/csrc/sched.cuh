@@ -12,6 +12,10 @@
 // (running max, running sum, unnormalised latent sum) into partial slot
 // 2w or 2w+1, which the combine step merges.
 //
+// When there are about as many row blocks as workers and they are of about
+// the same length (uniform decode), each worker takes one whole row block
+// instead, and nothing is split (see sched_kernel).
+//
 // Everything is integer arithmetic and deterministic: the split points depend
 // only on the lengths, never on the physical page order.
 #pragma once
@@ -35,7 +39,7 @@ struct Sched {
   int* worker_seg;    // [W+1]  first segment of each worker
   Seg* segs;          // [W+R]
   int* rb_seg_first;  // [R+1]  first segment of each row block
-  int* split_rbs;     // [2W+1] row blocks with more than one segment; [0] = count
+  int* split_rbs;     // [2W+1] first segment of each row block with more than one segment; [0] = count
 };
 
 struct SchedArgs {
@@ -125,12 +129,47 @@ __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
   const int R = a.R, W = a.W;
   const bool in_smem = R + 1 <= kSchedSmemRb;
   int* ts = in_smem ? sched_smem : a.s.tile_start;
-  for (int rb = tid; rb < R; rb += T)
+  __shared__ int longest;
+  if (tid == 0) longest = 0;
+  __syncthreads();
+  int my_longest = 0;
+  for (int rb = tid; rb < R; rb += T) {
     ts[rb] = ceil_div(rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, a.err), a.tile);
+    my_longest = max(my_longest, ts[rb]);
+  }
+  atomicMax(&longest, my_longest);
   __syncthreads();
   const int total = block_exclusive_scan(ts, R);
   if (tid == 0) ts[R] = total;
   __syncthreads();
+
+  // One whole row block per worker when there are nearly as many row blocks
+  // as workers (at least 7/8 of them) and none is more than 10% longer than
+  // the mean: nothing is split, so there are no partial results to combine
+  // and no worker changes query rows in mid-stream, which outweighs the at
+  // most 1/7 more pages per busy worker.  Workers past R get nothing.
+  if (R <= W && 8LL * R >= 7LL * W && 10LL * longest * R <= 11LL * total) {
+    int* wseg = a.s.worker_seg;
+    for (int w = tid; w <= W; w += T) wseg[w] = min(w, R);
+    for (int rb = tid; rb < R; rb += T) {
+      Seg g;
+      g.rb = rb;
+      g.t_lo = 0;
+      g.t_hi = ts[rb + 1] - ts[rb];
+      g.slot = -1;
+      g.nkeys = rb_nkeys(a.kv_len, a.uniform_kv_len, a.n_q, a.max_kv_len, rb, nullptr);
+      g.pad[0] = g.pad[1] = g.pad[2] = 0;
+      a.s.segs[rb] = g;
+      a.s.rb_seg_first[rb] = rb;
+    }
+    if (tid == 0) {
+      a.s.rb_seg_first[R] = R;
+      a.s.split_rbs[0] = 0;
+    }
+    if (in_smem)
+      for (int i = tid; i <= R; i += T) a.s.tile_start[i] = ts[i];
+    return;
+  }
 
   // Segment counts per worker.
   int* ws = a.s.worker_seg;
@@ -170,7 +209,8 @@ __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
     for (int i = tid; i <= R; i += T) a.s.tile_start[i] = ts[i];
   __syncthreads();
 
-  // Row blocks with more than one segment.  Such a row block starts with a
+  // Row blocks with more than one segment, by their first segment (their
+  // segments are consecutive in segs).  Such a row block starts with a
   // partial segment, which is the last segment of its worker; that worker
   // lists it (the order of the list does not affect any result).
   if (tid == 0) a.s.split_rbs[0] = 0;
@@ -179,7 +219,7 @@ __global__ void __launch_bounds__(1024) sched_kernel(SchedArgs a) {
     int s0 = ws[w], s1 = ws[w + 1];
     if (s1 > s0) {
       Seg g = a.s.segs[s1 - 1];
-      if (g.slot >= 0 && g.t_lo == 0) a.s.split_rbs[1 + atomicAdd(&a.s.split_rbs[0], 1)] = g.rb;
+      if (g.slot >= 0 && g.t_lo == 0) a.s.split_rbs[1 + atomicAdd(&a.s.split_rbs[0], 1)] = s1 - 1;
     }
   }
 }
