@@ -49,8 +49,9 @@ struct EpiStore {
 // Append: columns [0, d_c) are the latent, [d_c, d_cr) the position key (one
 // shared key of d_r, or one per head), every d_r-wide key rotated by the
 // token's position, then the row goes to its cache slot.
-// Without seq_idx/pos (prefill), row m is token m % prefill_S of sequence
-// m / prefill_S.
+// Without seq_idx/pos, row m is either token m % prefill_S of sequence
+// m / prefill_S (prefill) or, with kv_len, new token q = m % n_q of sequence
+// b = m / n_q at position kv_len[b] - n_q + q (a decode step).
 template <typename OutT>
 struct EpiAppend {
   OutT* cache;
@@ -63,15 +64,23 @@ struct EpiAppend {
   int d_r;                 // RoPE-key width: columns [d_c, d_cr) are one key or n_h keys of d_r each
   int* err;
   OutT* dense;             // optional: every row also at dense[m * d_cr] (token order), else null
-  __device__ void operator()(int, int m, int n, float v0, float v1) const {
-    int s, p;
+  const int32_t* kv_len;   // decode step: lengths after the append, and
+  int n_q;                 // new tokens per sequence
+  __device__ void locate(int m, int& s, int& p) const {
     if (seq_idx) {
       s = seq_idx[m];
       p = pos[m];
+    } else if (kv_len) {
+      s = m / n_q;
+      p = kv_len[s] - n_q + (m - s * n_q);
     } else {
       s = m / prefill_S;
       p = m - s * prefill_S;
     }
+  }
+  __device__ void operator()(int, int m, int n, float v0, float v1) const {
+    int s, p;
+    locate(m, s, p);
     if (s < 0 || s >= n_seq || p < 0 || p >= max_pages * page_size) {
       flag_error(err, kErrBounds);
       return;
@@ -89,13 +98,7 @@ struct EpiAppend {
   // the eight are all latent or all position key).
   __device__ void store8(int, int m, int n0, const float (&v)[8]) const {
     int s, p;
-    if (seq_idx) {
-      s = seq_idx[m];
-      p = pos[m];
-    } else {
-      s = m / prefill_S;
-      p = m - s * prefill_S;
-    }
+    locate(m, s, p);
     if (s < 0 || s >= n_seq || p < 0 || p >= max_pages * page_size) {
       flag_error(err, kErrBounds);
       return;

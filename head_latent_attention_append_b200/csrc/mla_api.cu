@@ -60,6 +60,8 @@ void prof_mark(cudaStream_t st, bool start) {
 constexpr int kWorkerSlots = 296;        // partial-slot capacity: 2 * kWorkerSlots
 constexpr int kSplitKTileSplits = 1024;  // split-K scratch: tiles * splits <= this
 constexpr int kCounterCap = 1024;
+constexpr int kSideTileSplits = 256;     // split-K scratch of the side-stream append (tiles * splits)
+constexpr int kSideAppendCtas = 32;      // CTAs of the side-stream append GEMM
 constexpr double kLog2e = 1.4426950408889634074;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -189,12 +191,14 @@ WeightLayout weight_layout(const mla_dims& d) {
 // Workspace layout shared by the size queries and the calls.
 struct Plan {
   size_t hdr, counters, partial, cq, qc, qabs, tile_start, worker_seg, segs, rb_first, split_rbs,
-      part_o, part_ml, obar, total;
+      part_o, part_ml, obar, side_partial, total;
   int R, qrows;
 };
 // cp: context-parallel partials, where every segment (at most W + R) has its
 // own partial slot.
-Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false) {
+// side_append: the split-K scratch of an append GEMM that runs on the side
+// stream beside the query projections (a decode step).
+Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false, bool side_append = false) {
   const size_t e = esize(d);
   Plan P{};
   P.R = R;
@@ -217,6 +221,9 @@ Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false) {
     P.part_o = o;     o = align_up(o + e * slots * d.n_h * d.d_c, 256);
     P.part_ml = o;    o = align_up(o + sizeof(float) * slots * 2 * d.n_h * 2, 256);
     P.obar = o;       o = align_up(o + e * (size_t)R * d.n_h * d.d_c, 256);
+  }
+  if (side_append) {
+    P.side_partial = o; o = align_up(o + sizeof(float) * (size_t)kSideTileSplits * 64 * 64, 256);
   }
   P.total = o;
   return P;
@@ -323,7 +330,7 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, long long dim0, long lon
 template <int BN, class Epi>
 cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                            int M, int N, int K, int batch, const Epi& epi, float* partial, long long partial_floats,
-                           cudaStream_t st) {
+                           cudaStream_t st, int max_ctas) {
   CUtensorMap mapW, mapX;
   // Weights: batches are contiguous row blocks of N rows.
   if (batch > 1 && sB != (long long)N * ldb) return cudaErrorInvalidValue;
@@ -340,7 +347,7 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   // keep every SM streaming weights; the reduce kernel sums the splits in
   // order and runs the epilogue.
   int splits = 1;
-  const int sms = num_sms();
+  const int sms = std::min(num_sms(), max_ctas);
   if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), ceil_div(2 * sms, tiles));
   while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
   const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
@@ -368,16 +375,20 @@ cudaError_t gemm_simt(const void* A, long long lda, long long sA, const void* B,
                       int N, int K, int batch, const Epi& epi, void* ws, const Plan& P, cudaStream_t st,
                       int tile_split_cap);
 
+// `max_ctas` caps the CTAs of the tensor-core GEMM (a GEMM sharing the GPU
+// with another stream's).
 template <typename T, class Epi>
 cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                  int M, int N, int K, int batch, const Epi& epi, void* ws, const Plan& P,
-                 cudaStream_t st, int tile_split_cap = kSplitKTileSplits) {
+                 cudaStream_t st, int tile_split_cap = kSplitKTileSplits, int max_ctas = INT_MAX) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if constexpr (sizeof(T) == 2) {
     const long long cap = (long long)tile_split_cap * 64 * 64;
     if (M <= 512)
-      return gemm_tc_launch<64>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st);
-    return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st);
+      return gemm_tc_launch<64>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
+                                max_ctas);
+    return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
+                               max_ctas);
   } else {
     return gemm_simt(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, ws, P, st, tile_split_cap);
   }
@@ -416,16 +427,22 @@ cudaError_t gemm_simt(const void* A, long long lda, long long sA, const void* B,
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // ------------------------------------------------------------- pipelines
+// kv_len (decode step): token m is new token m % n_q of sequence m / n_q, at
+// position kv_len[b] - n_q + q.
 template <typename T>
 mla_status append_impl(const mla_weights* w, const void* h, const int32_t* seq_idx, const int32_t* pos,
                        int prefill_S, int n_seq, const int32_t* page_table, int max_pages, int num_pages,
-                       void* cache, int T_, void* ws, const Plan& P, cudaStream_t st) {
+                       void* cache, int T_, void* ws, const Plan& P, cudaStream_t st,
+                       const int32_t* kv_len = nullptr, int n_q = 0, int tile_split_cap = kSplitKTileSplits,
+                       int max_ctas = INT_MAX) {
   const mla_dims& d = w->d;
   EpiAppend<T> epi{};
   epi.cache = static_cast<T*>(cache);
   epi.seq_idx = seq_idx;
   epi.pos = pos;
   epi.prefill_S = prefill_S;
+  epi.kv_len = kv_len;
+  epi.n_q = n_q;
   epi.page_table = page_table;
   for (int i = 0; i < d.d_r / 2; ++i) epi.theta[i] = w->theta[i];
   epi.max_pages = max_pages;
@@ -437,7 +454,7 @@ mla_status append_impl(const mla_weights* w, const void* h, const int32_t* seq_i
   epi.n_seq = n_seq;
   epi.err = at<int>(ws, P.hdr);
   return cuda_status(gemm<T>(h, d.d_model, 0, w->dkr, d.d_model, 0, T_, cache_row(d), d.d_model, 1, epi,
-                             ws, P, st));
+                             ws, P, st, tile_split_cap, max_ctas));
 }
 
 // Context-parallel partial: the rank's window and where its (obar_r, lse_r)
@@ -448,11 +465,18 @@ struct CpOut {
   float* lse;  // [R][n_h]
 };
 
+// A decode step's append, run on the side stream beside the query
+// projections: the new tokens' rows (h, one per row block) into `cache`.
+struct SideAppend {
+  void* cache;
+  int n_seq;
+};
+
 template <typename T>
 mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_len, int uniform_kv_len,
                        int n_q, int prefill_S, const int32_t* page_table, int max_pages, int num_pages,
                        const void* cache, float* out, int R, int max_kv_len, void* ws, const Plan& P,
-                       cudaStream_t st, const CpOut* cp = nullptr) {
+                       cudaStream_t st, const CpOut* cp = nullptr, const SideAppend* side_append = nullptr) {
   const mla_dims& d = w->d;
   const int q_row = d.d_c + d.d_r;  // a Q_abs row: [q~ | q_R]
   const int d_cr = cache_row(d);    // a cache row: [c | k_R] (one key or n_h)
@@ -507,7 +531,18 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
       if ((e = set_smem_once(sched_kernel, sizeof(int) * (size_t)kSchedSmemRb))) return cuda_status(e);
       sched_kernel<<<1, 512, sched_smem, side->s>>>(sa);
     }
-    if ((e = cudaGetLastError()) || (e = cudaEventRecord(side->join, side->s))) return cuda_status(e);
+    if ((e = cudaGetLastError())) return cuda_status(e);
+    if (side_append) {
+      // The append GEMM on a share of the SMs, with its own split-K scratch
+      // (the query projections' splits use P.partial at the same time).
+      Plan Ps = P;
+      Ps.partial = P.side_partial;
+      const mla_status s = append_impl<T>(w, hq, nullptr, nullptr, 0, side_append->n_seq, page_table, max_pages,
+                                          num_pages, side_append->cache, R, ws, Ps, side->s, kv_len, n_q,
+                                          kSideTileSplits, kSideAppendCtas);
+      if (s != MLA_OK) return s;
+    }
+    if ((e = cudaEventRecord(side->join, side->s))) return cuda_status(e);
   }
   // (1) query latent.
   const void* src = hq;
@@ -888,6 +923,38 @@ mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_l
     return attend_impl<__nv_bfloat16>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out,
                                       B * n_q, max_kv_len, workspace, P, stream);
   return attend_impl<float>(w, h_q, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out, B * n_q,
+                            max_kv_len, workspace, P, stream);
+}
+
+size_t mla_decode_step_workspace_bytes(const mla_dims* dims, int B, int n_q, int max_kv_len) {
+  if (check_dims(dims) != MLA_OK || B <= 0 || n_q <= 0 || max_kv_len < n_q) return 0;
+  return make_plan(*dims, B * n_q, true, false, true).total;
+}
+
+mla_status mla_decode_step(const mla_weights* w, const void* h, const int32_t* kv_len, const int32_t* page_table,
+                           int max_pages, int num_pages, void* cache, float* out, int B, int n_q, int max_kv_len,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!w || B <= 0 || n_q <= 0 || max_kv_len < n_q || max_pages <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!h || !kv_len || !page_table || !cache || !out || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)max_pages * w->d.page_size < max_kv_len) return MLA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(h, 16) || !aligned(cache, 16) || !aligned(out, 16))
+    return MLA_ERR_INVALID_ARG;
+  const Plan P = make_plan(w->d, B * n_q, true, false, true);
+  if (workspace_bytes < P.total) return MLA_ERR_WORKSPACE;
+  mla_status s = begin_call(workspace, stream, P);
+  if (s != MLA_OK) return s;
+  if (w->d.dtype == MLA_BF16) {
+    const SideAppend sa{cache, B};
+    return attend_impl<__nv_bfloat16>(w, h, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out,
+                                      B * n_q, max_kv_len, workspace, P, stream, nullptr, &sa);
+  }
+  // fp32: the CUDA-core GEMMs share one arrival-counter array, so the append
+  // runs first on the caller's stream.
+  s = append_impl<float>(w, h, nullptr, nullptr, 0, B, page_table, max_pages, num_pages, cache, B * n_q, workspace,
+                         P, stream, kv_len, n_q);
+  if (s != MLA_OK) return s;
+  return attend_impl<float>(w, h, kv_len, 0, n_q, 0, page_table, max_pages, num_pages, cache, out, B * n_q,
                             max_kv_len, workspace, P, stream);
 }
 

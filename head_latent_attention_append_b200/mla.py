@@ -27,6 +27,7 @@ EXPORTED = [
     "mla_last_launch_count", "mla_profile_begin", "mla_profile_end", "mla_append_latent_noalloc",
     "mla_decode_cp_workspace_bytes", "mla_decode_cp_partial", "mla_decode_cp_combine",
     "mla_selftest_wait_timeout", "mla_prefill_materialised_workspace_bytes", "mla_prefill_materialised",
+    "mla_decode_step_workspace_bytes", "mla_decode_step",
 ]
 APPEND_NOALLOC_MAX_T = 256
 
@@ -65,6 +66,8 @@ def _load():
         "mla_append_latent": (S, [P, P, P, P, P, I, I, I, P, I, P, Z, P]),
         "mla_decode_workspace_bytes": (Z, [D, I, I, I]),
         "mla_decode": (S, [P, P, P, P, I, I, P, P, I, I, I, P, Z, P]),
+        "mla_decode_step_workspace_bytes": (Z, [D, I, I, I]),
+        "mla_decode_step": (S, [P, P, P, P, I, I, P, P, I, I, I, P, Z, P]),
         "mla_prefill_workspace_bytes": (Z, [D, I, I]),
         "mla_prefill": (S, [P, P, P, I, I, P, P, I, I, P, Z, P]),
         "mla_get_error": (S, [P, P]),
@@ -116,6 +119,10 @@ def append_workspace_bytes(dims: Dims, T: int) -> int:
 
 def decode_workspace_bytes(dims: Dims, B: int, n_q: int, max_kv_len: int) -> int:
     return lib.mla_decode_workspace_bytes(ctypes.byref(dims), B, n_q, max_kv_len)
+
+
+def decode_step_workspace_bytes(dims: Dims, B: int, n_q: int, max_kv_len: int) -> int:
+    return lib.mla_decode_step_workspace_bytes(ctypes.byref(dims), B, n_q, max_kv_len)
 
 
 def prefill_workspace_bytes(dims: Dims, B: int, S: int) -> int:
@@ -190,6 +197,16 @@ def decode(w: Weights, h_q, kv_len, page_table, num_pages: int, cache, out, max_
     B, n_q = h_q.shape[0], h_q.shape[1]
     _check("mla_decode", lib.mla_decode(
         w.handle, _ptr(h_q), _ptr(kv_len), _ptr(page_table), page_table.shape[1], num_pages, _ptr(cache),
+        _ptr(out), B, n_q, max_kv_len, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def decode_step(w: Weights, h, kv_len, page_table, num_pages: int, cache, out, max_kv_len: int, workspace,
+                stream=None):
+    """Append the new tokens' latent rows, then decode them (one call)."""
+    B, n_q = h.shape[0], h.shape[1]
+    _check("mla_decode_step", lib.mla_decode_step(
+        w.handle, _ptr(h), _ptr(kv_len), _ptr(page_table), page_table.shape[1], num_pages, _ptr(cache),
         _ptr(out), B, n_q, max_kv_len, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
 

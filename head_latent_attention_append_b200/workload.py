@@ -160,20 +160,26 @@ def setup(name: str, device="cuda", checked_count: int = 4, check_all: Optional[
     if ws_app is None or ws_app.numel() < need:
         ws_app = torch.empty(need, dtype=torch.uint8, device=dev)
     out = torch.empty((wl.B, wl.n_q, wl.n_h, wl.d_v), dtype=torch.float32, device=dev)
-    ws = torch.empty(mla.decode_workspace_bytes(dims, wl.B, wl.n_q, int(kv.max())), dtype=torch.uint8, device=dev)
+    ws = torch.empty(mla.decode_step_workspace_bytes(dims, wl.B, wl.n_q, int(kv.max())), dtype=torch.uint8,
+                     device=dev)
     return Setup(wl, dims, hw, weights, kv, layout, kv_len, page_table, cache, h_new, seq_idx, pos, out, ws_app,
                  ws, checked, host_hidden)
 
 
-def step(s: Setup, stream=None) -> int:
-    """One pass of the hot path: append the new tokens, then attend (decode),
-    or append every token and attend causally (prefill).  Returns the number
-    of kernels libmla launched."""
+def step(s: Setup, stream=None, fused: bool = True) -> int:
+    """One pass of the hot path: append the new tokens, then attend (decode:
+    one mla_decode_step call, or with fused=False mla_append_latent then
+    mla_decode), or append every token and attend causally (prefill).  Returns
+    the number of kernels libmla launched."""
     if s.wl.mode == "prefill":
         fn = mla.prefill_materialised if s.wl.materialised else mla.prefill
         fn(s.weights, s.h_new, s.page_table, s.layout.num_pages, s.cache, s.out, s.ws, stream)
         return mla.last_launch_count()
     wl = s.wl
+    if fused:
+        mla.decode_step(s.weights, s.h_new, s.kv_len, s.page_table, s.layout.num_pages, s.cache, s.out,
+                        s.max_kv_len, s.ws, stream)
+        return mla.last_launch_count()
     mla.append_latent(s.weights, s.h_new.view(wl.B * wl.n_q, wl.d_model), s.seq_idx, s.pos, s.page_table,
                       s.layout.num_pages, s.cache, s.ws_append, stream)
     n = mla.last_launch_count()

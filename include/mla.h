@@ -198,6 +198,30 @@ mla_status mla_decode(const mla_weights* w, const void* h_q, const int32_t* kv_l
                       size_t workspace_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Decode step: append, then decode, in one call.  The same computation as
+ * mla_append_latent of the n_q new tokens of every sequence (token q of
+ * sequence b at position kv_len[b]-n_q+q, its rows of h as the hidden
+ * states) followed by mla_decode with h_q = h: c_KV = W_DKV h and
+ * k_R = RoPE(W_KR h) go into `cache` ("ai-decoupled-rope-mla", the cached
+ * latent and the decoupled key), then the new tokens attend as in
+ * mla_decode.  Outputs and cache rows are bit-identical to the two calls.
+ *   - h: [B, n_q, d_model] hidden states of the new tokens.
+ *   - kv_len [B] (device): keys per sequence including the new tokens;
+ *     page_table must map their positions.
+ *   - cache is written (the new rows) and read.
+ * With bf16 the append's GEMM runs on the library's side stream (forked from
+ * and joined back into `stream` inside the call, as the schedule does) on a
+ * share of the SMs, beside the query projections, so it costs little of the
+ * step.  Workspace: mla_decode_step_workspace_bytes(...) (the decode
+ * workspace plus the append's own split-K scratch).
+ * ------------------------------------------------------------------------- */
+size_t mla_decode_step_workspace_bytes(const mla_dims* dims, int B, int n_q, int max_kv_len);
+mla_status mla_decode_step(const mla_weights* w, const void* h, const int32_t* kv_len,
+                           const int32_t* page_table, int max_pages, int num_pages, void* cache,
+                           float* out, int B, int n_q, int max_kv_len, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Context-parallel decode: one sequence's cache spread over several ranks
  * (GPUs).  The pages do not split a sequence over devices; the split rests
  * on the identity that the softmax denominators of disjoint key sets add up

@@ -365,3 +365,49 @@ def test_per_head_rope_keys_full_size_match_oracle():
     assert mla.get_error(s.ws) == mla.MLA_OK
     err = check_decode(s, TOL["bf16"])
     print(f"per-head RoPE keys: max rel err {err:.3e}")
+
+@pytest.mark.parametrize("n_q", [1, 3])
+def test_decode_step_equals_append_then_decode(n_q):
+    """mla_decode_step (the append on the side stream beside the query
+    projections) writes the same cache rows and outputs, bit for bit, as
+    mla_append_latent of the new tokens followed by mla_decode."""
+    mla, _ = _mods()
+    c = small_case([0, 1, 63, 64, 300, 1000], n_q)
+    wl, dev, dt, lay = c["wl"], c["dev"], c["dt"], c["lay"]
+    pt = torch.from_numpy(lay.page_table).to(dev)
+    kv = c["kv"]
+    # History (every token but the new ones) appended into one cache; two copies of it.
+    T = int((kv - n_q).sum())
+    base = torch.full((lay.num_pages, 64, wl.d_cr), float("nan"), dtype=dt, device=dev)
+    if T:
+        h = torch.from_numpy(np.concatenate([c["H"][b][:int(L) - n_q] for b, L in enumerate(kv)])).to(dev, dt)
+        si = torch.from_numpy(np.concatenate([np.full(int(L) - n_q, b, np.int32) for b, L in enumerate(kv)])).to(dev)
+        ps = torch.from_numpy(np.concatenate([np.arange(int(L) - n_q, dtype=np.int32) for L in kv])).to(dev)
+        wsa = torch.empty(mla.append_workspace_bytes(c["dims"], T), dtype=torch.uint8, device=dev)
+        mla.append_latent(c["weights"], h, si, ps, pt, lay.num_pages, base, wsa)
+    cache_a, cache_b = base.clone(), base.clone()
+    hq = torch.from_numpy(np.stack([c["H"][b][-n_q:] for b in range(wl.B)])).to(dev, dt)
+    kvd = torch.from_numpy(kv).to(dev)
+    maxkv = int(kv.max())
+    # Two calls.
+    si = torch.arange(wl.B, dtype=torch.int32, device=dev).repeat_interleave(n_q)
+    ps = torch.from_numpy(np.concatenate([np.arange(int(L) - n_q, int(L)) for L in kv]).astype(np.int32)).to(dev)
+    wsa = torch.empty(mla.append_workspace_bytes(c["dims"], wl.B * n_q), dtype=torch.uint8, device=dev)
+    mla.append_latent(c["weights"], hq.view(wl.B * n_q, -1), si, ps, pt, lay.num_pages, cache_a, wsa)
+    out_a = torch.empty((wl.B, n_q, wl.n_h, wl.d_v), dtype=torch.float32, device=dev)
+    ws = torch.empty(mla.decode_workspace_bytes(c["dims"], wl.B, n_q, maxkv), dtype=torch.uint8, device=dev)
+    mla.decode(c["weights"], hq, kvd, pt, lay.num_pages, cache_a, out_a, maxkv, ws)
+    # One call.
+    out_b = torch.empty_like(out_a)
+    wss = torch.empty(mla.decode_step_workspace_bytes(c["dims"], wl.B, n_q, maxkv), dtype=torch.uint8, device=dev)
+    mla.decode_step(c["weights"], hq, kvd, pt, lay.num_pages, cache_b, out_b, maxkv, wss)
+    torch.cuda.synchronize()
+    assert mla.get_error(ws) == 0 and mla.get_error(wss) == 0 and mla.get_error(wsa) == 0
+    assert torch.equal(torch.nan_to_num(cache_a, nan=7.0), torch.nan_to_num(cache_b, nan=7.0))
+    assert torch.equal(out_a, out_b)
+    # And against the oracle.
+    dims = oracle_dims(wl)
+    w = O.Weights(**c["hw"].as_dict())
+    got = out_b.cpu().numpy()
+    for b in range(wl.B):
+        assert rel_err(got[b], O.mla_decode(dims, w, c["H"][b], n_q)) <= TOL["bf16"]
