@@ -585,7 +585,7 @@ def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
 # paged decode.
 EXTRA = {"prefill": "dsv2_bf16_prefill", "ragged": "dsv2_ragged_decode",
          "prefill_materialised": "dsv2_bf16_prefill_mat", "page": "page_bf16_decode",
-         "page_per_head_rope": "page_bf16_decode_rph"}
+         "page_per_head_rope": "page_bf16_decode_rph", "spec4": "dsv2_spec4_decode"}
 
 
 def run_ours(args):
