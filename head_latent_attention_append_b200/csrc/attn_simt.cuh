@@ -37,6 +37,12 @@ struct AttnArgs {
   float* part_ml;            // [2W][2][n_h][2]: (m, l) per latent-column half (ml_index)
   void* obar;                // [R][n_h][d_c] (type of the path)
   int* err;
+  // Arrival counters [R][2] (zero at the start of a call), or null.  With
+  // them the tensor-core kernel merges a split row block itself: each piece
+  // counts in after writing its partial slot, and the last of a CTA rank's
+  // pieces merges all of them (in segment order) into obar; no combine
+  // kernel runs.
+  int* arrive;
 };
 
 // Index into part_ml of the (m, l) pair of partial slot `slot`, latent-column

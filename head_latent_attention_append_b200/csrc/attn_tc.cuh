@@ -78,6 +78,7 @@ constexpr int CH_V = KT * 128;            // 64 keys x 64 bf16 columns (8 KB)
 constexpr int MAX_NK = 9;                 // 64-column chunks of a cache row (d_c <= 512, d_r <= 64)
 constexpr int MAX_NPV = 4;                // latent chunks per CTA (d_c / 128)
 constexpr int MAX_TS = 6;                 // chunks of Q held in TMEM
+constexpr int MAX_PIECES = 80;            // pieces of a split row block merged in the kernel (<= workers)
 constexpr int SGS = 3, VGS = 2;           // ring slots
 constexpr int SG_BYTES = MAX_NK * CH_S;   // 36 KB
 constexpr int VG_BYTES = MAX_NPV * CH_V;  // 32 KB
@@ -648,6 +649,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         constexpr int PPR = 4 * NPV;          // 16-byte pieces per staged row
         constexpr int SROW = 16 * PPR + 16;   // padded row: consecutive rows start in different banks
         static_assert(64 * SROW <= 2 * P_BYTES + CH_V, "staged output fits the P and staging tiles");
+        static_assert((HEADS + 1) * MAX_PIECES * 4 <= 2 * P_BYTES + CH_V, "merge weights fit the P and staging tiles");
         uint8_t* const so = smem + OFF_P;
         __nv_bfloat16* const obase = whole ? static_cast<__nv_bfloat16*>(a.obar) + (long long)g.rb * a.n_h * a.d_c
                                            : static_cast<__nv_bfloat16*>(a.part_o) + (long long)g.slot * a.n_h * a.d_c;
@@ -687,6 +689,110 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             float* ml = a.part_ml + ml_index(g.slot, half, a.n_h, head);
             ml[0] = m_used;
             ml[1] = lrow;
+          }
+        }
+        if (a.arrive && !whole) {
+          // A piece of a split row block counts in; the last piece of this
+          // CTA rank to do so merges all of them, read back from their slots
+          // in segment order, so the result does not depend on which piece
+          // came last:
+          //   w_k = 2^(m_k - max_j m_j) l_k,  obar = sum_k w_k N_k / sum_k w_k
+          // (N_k the piece's normalised rows).  One thread publishes the
+          // CTA's slot writes (barrier, fence, atomic) and, if last, fences
+          // again before the others read the other pieces' slots.
+          volatile int* const merge_info = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);  // np or 0, sb
+          named_bar_sync(3, 256);
+          if (tid == 128) {
+            const int sb = a.sched.rb_seg_first[g.rb], se = a.sched.rb_seg_first[g.rb + 1];
+            __threadfence();
+            const int old = ok ? atomicAdd(a.arrive + 2 * g.rb + (int)rank, 1) : -1;
+            const bool last = old == se - sb - 1;
+            if (last) __threadfence();
+            merge_info[0] = last ? se - sb : 0;
+            merge_info[1] = sb;
+          }
+          named_bar_sync(3, 256);
+          const int np = merge_info[0];
+          if (np > 0) {
+            const int sb = merge_info[1];
+            float* const coef = reinterpret_cast<float*>(smem + OFF_P);  // [HEADS][MAX_PIECES] w_k / sum w
+            int* const slot_of = reinterpret_cast<int*>(coef + HEADS * MAX_PIECES);
+            const int u = tid - 128;
+            for (int k = u; k < np; k += 256) slot_of[k] = __ldg(&segs[sb + k].slot);
+            if (u < HEADS && (int)rank * HEADS + u < a.n_h) {
+              // One pass over the pieces' (m_k, l_k), four in flight:
+              // e_k = m_k + log2 l_k (l_k >= 1: a piece holds its own
+              // maximum), then w_k = 2^(e_k - m) from shared memory.
+              const int hd = (int)rank * HEADS + u;
+              float m = -INFINITY;
+              for (int k0 = 0; k0 < np; k0 += 4) {
+                int sl[4];
+                float2 mlk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sl[i] = k0 + i < np ? __ldg(&segs[sb + k0 + i].slot) : -1;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  mlk[i] = sl[i] >= 0 ? __ldcg(reinterpret_cast<const float2*>(a.part_ml + ml_index(sl[i], 0, a.n_h, hd)))
+                                      : make_float2(-INFINITY, 1.f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  m = fmaxf(m, mlk[i].x);
+                  if (k0 + i < np) coef[u * MAX_PIECES + k0 + i] = mlk[i].x + __log2f(mlk[i].y);
+                }
+              }
+              float l = 0.f;
+              for (int k = 0; k < np; ++k) l += exp2f(coef[u * MAX_PIECES + k] - m);
+              const float il = 1.f / l;
+              for (int k = 0; k < np; ++k) coef[u * MAX_PIECES + k] = exp2f(coef[u * MAX_PIECES + k] - m) * il;
+            }
+            named_bar_sync(3, 256);
+            // GM sixteen-byte pieces of output per thread at a time, the GM
+            // loads of one partial slot in flight together.
+            constexpr int PPR = 16 * NPV;  // 16-byte pieces per row
+            constexpr int GM = 4 * NPV % 8 == 0 ? 8 : (4 * NPV < 8 ? 4 * NPV : 2 * NPV);
+            static_assert(HEADS * PPR % (256 * GM) == 0, "whole groups of pieces per thread");
+            __nv_bfloat16* const orow = static_cast<__nv_bfloat16*>(a.obar) + (long long)g.rb * a.n_h * a.d_c;
+            const __nv_bfloat16* const pbase = static_cast<const __nv_bfloat16*>(a.part_o);
+            const long long slot_elems = (long long)a.n_h * a.d_c;
+#pragma unroll 1
+            for (int gi = 0; gi < HEADS * PPR / 256; gi += GM) {
+              int off[GM], cr[GM];
+              float acc[GM][8];
+#pragma unroll
+              for (int i = 0; i < GM; ++i) {
+                const int x = u + 256 * (gi + i), r = x / PPR, hd = (int)rank * HEADS + r;
+                off[i] = hd < a.n_h ? hd * a.d_c + 8 * (x - r * PPR) : -1;
+                cr[i] = r * MAX_PIECES;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+              }
+#pragma unroll 1
+              for (int k = 0; k < np; ++k) {
+                const __nv_bfloat16* const src = pbase + slot_of[k] * slot_elems;
+                uint4 v[GM];
+#pragma unroll
+                for (int i = 0; i < GM; ++i)
+                  v[i] = off[i] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(src + off[i])) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < GM; ++i) {
+                  const float c = coef[cr[i] + k];
+                  const uint32_t vw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vw[q]));
+                    acc[i][2 * q] = __fmaf_rn(c, f.x, acc[i][2 * q]);
+                    acc[i][2 * q + 1] = __fmaf_rn(c, f.y, acc[i][2 * q + 1]);
+                  }
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < GM; ++i)
+                if (ok && off[i] >= 0)
+                  *reinterpret_cast<uint4*>(orow + off[i]) =
+                      make_uint4(pack_bf16x2(acc[i][0], acc[i][1]), pack_bf16x2(acc[i][2], acc[i][3]),
+                                 pack_bf16x2(acc[i][4], acc[i][5]), pack_bf16x2(acc[i][6], acc[i][7]));
+            }
+            named_bar_sync(3, 256);  // shared memory is the next segment's again
           }
         }
         if (ok) {

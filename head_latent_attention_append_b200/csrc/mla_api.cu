@@ -190,7 +190,7 @@ WeightLayout weight_layout(const mla_dims& d) {
 
 // Workspace layout shared by the size queries and the calls.
 struct Plan {
-  size_t hdr, counters, partial, cq, qc, qabs, tile_start, worker_seg, segs, rb_first, split_rbs,
+  size_t hdr, counters, arrive, partial, cq, qc, qabs, tile_start, worker_seg, segs, rb_first, split_rbs,
       part_o, part_ml, obar, side_partial, total;
   int R, qrows;
 };
@@ -208,6 +208,9 @@ Plan make_plan(const mla_dims& d, int R, bool attention, bool cp = false, bool s
   size_t o = 0;
   P.hdr = o;        o = align_up(o + 256, 256);
   P.counters = o;   o = align_up(o + sizeof(int) * kCounterCap, 256);
+  // Arrival counters of split row blocks per CTA rank, zeroed with the
+  // header and the split-K counters at the start of every call.
+  P.arrive = o;     o = align_up(o + sizeof(int) * (attention ? 2 * (size_t)R : 0), 256);
   P.partial = o;    o = align_up(o + sizeof(float) * (size_t)kSplitKTileSplits * 64 * 64, 256);
   if (attention) {
     P.cq = o;         o = align_up(o + e * (size_t)R * d.d_cq, 256);
@@ -519,6 +522,11 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
   int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
                        : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
+  // bf16 without context parallelism: the attention kernel merges split row
+  // blocks itself (a row block has at most one piece per worker), and no
+  // combine kernel runs.
+  const bool self_merge = kTensorCores && !cp && W <= attn_tc::MAX_PIECES;
+  if (self_merge) aa.arrive = at<int>(ws, P.arrive);
   {
     SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};
     ++g_launches;
@@ -611,7 +619,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     cp_combine_kernel<T><<<dim3(R, ceil_div(d.n_h, 8)), 256, 0, st>>>(aa, static_cast<T*>(cp->obar), cp->lse);
     return cuda_status(cudaGetLastError());
   }
-  {
+  if (!self_merge) {
     ++g_launches;
     if ((e = launch_pdl(combine_kernel<T>, dim3(2 * W, ceil_div(d.n_h, 8)), dim3(256), 0, st, aa)))
       return cuda_status(e);
@@ -744,7 +752,7 @@ __global__ void wait_timeout_kernel(int* err, unsigned long long limit_ns) {
 
 mla_status begin_call(void* ws, cudaStream_t st, const Plan& P) {
   g_launches = 0;
-  return cuda_status(cudaMemsetAsync(ws, 0, P.partial, st));  // header + split-K counters
+  return cuda_status(cudaMemsetAsync(ws, 0, P.partial, st));  // header, split-K and arrival counters
 }
 
 }  // namespace

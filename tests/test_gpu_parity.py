@@ -190,6 +190,22 @@ def test_two_runs_are_bitwise_identical():
     np.testing.assert_array_equal(a, b)
 
 
+@pytest.mark.parametrize("lengths,n_q", [([9000], 1), ([9000, 5], 2)])
+def test_one_long_row_block_split_over_every_worker_matches_oracle(lengths, n_q):
+    """One long sequence: its row blocks are cut into a piece per worker (one
+    per CTA pair), and the last piece of each to finish merges them all."""
+    c = small_case(lengths, n_q)
+    out, _, e1, e2 = run_small(c)
+    assert e1 == 0 and e2 == 0
+    dims = oracle_dims(c["wl"])
+    w = O.Weights(**c["hw"].as_dict())
+    for b in range(len(lengths)):
+        ref = O.mla_decode(dims, w, c["H"][b], n_q)
+        assert rel_err(out[b], ref) <= TOL["bf16"], b
+    again, _, _, _ = run_small(c)
+    np.testing.assert_array_equal(out, again)
+
+
 @pytest.mark.parametrize("n_q,j", [(2, 1), (4, 2)])
 def test_later_new_token_does_not_reach_earlier_query(n_q, j):
     mla, _ = _mods()
