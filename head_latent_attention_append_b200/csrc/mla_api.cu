@@ -522,10 +522,13 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
   int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
                        : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
-  // bf16 without context parallelism: the attention kernel merges split row
-  // blocks itself (a row block has at most one piece per worker), and no
-  // combine kernel runs.
-  const bool self_merge = kTensorCores && !cp && W <= attn_tc::MAX_PIECES;
+  // bf16 without context parallelism, with at least half as many row blocks
+  // as workers (so a split row block has two or three pieces): the attention
+  // kernel merges split row blocks itself (a row block has at most one piece
+  // per worker), and no combine kernel runs.  With fewer row blocks each has
+  // many pieces, all ending together, and the combine kernel spreads their
+  // merge over every SM instead.
+  const bool self_merge = kTensorCores && !cp && W <= attn_tc::MAX_PIECES && 2 * R >= W;
   if (self_merge) aa.arrive = at<int>(ws, P.arrive);
   {
     SchedArgs sa{kv_len, uniform_kv_len, n_q, R, W, d.page_size, max_kv_len, S, err};

@@ -190,10 +190,12 @@ def test_two_runs_are_bitwise_identical():
     np.testing.assert_array_equal(a, b)
 
 
-@pytest.mark.parametrize("lengths,n_q", [([9000], 1), ([9000, 5], 2)])
+@pytest.mark.parametrize("lengths,n_q", [([9000], 1), ([9000, 5], 2), ([100] * 19 + [20000], 2)])
 def test_one_long_row_block_split_over_every_worker_matches_oracle(lengths, n_q):
     """One long sequence: its row blocks are cut into a piece per worker (one
-    per CTA pair), and the last piece of each to finish merges them all."""
+    per CTA pair).  With few row blocks the combine kernel merges the pieces;
+    with 40 (at least half as many as workers) the attention kernel's last
+    piece of each row block merges them all, here 30-odd pieces."""
     c = small_case(lengths, n_q)
     out, _, e1, e2 = run_small(c)
     assert e1 == 0 and e2 == 0
