@@ -219,8 +219,8 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float
 
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(AttnArgs a) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial slots come from the attention kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const Sched& S = a.sched;
   const int idx = blockIdx.x;
   const int W = gridDim.x >> 1;

@@ -190,7 +190,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   constexpr int NSS = NK - NTS;                      // chunks of Q in shared memory
   static_assert(NPV >= 1 && NPV <= MAX_NPV && NSS * CH_V <= QS_BYTES, "latent width");
   extern __shared__ __align__(1024) uint8_t smem[];
-  pdl_trigger();
   if (smem_u32(smem) & 1023u) {  // the same in every CTA: all leave before any barrier
     if (threadIdx.x == 0) flag_error(a.err, kErrLayout);
     return;
@@ -250,6 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   // Everything above overlaps the previous kernel's tail; the schedule and
   // Q_abs come from earlier kernels.
   pdl_wait();
+  pdl_trigger();  // only now: a successor may read its weights before its own wait
   const Seg* segs = a.sched.segs;
   const int seg_lo = a.sched.worker_seg[w], seg_hi = a.sched.worker_seg[w + 1];
 

@@ -30,6 +30,10 @@ struct Args {
   int b_is_3d;               // B map has a per-batch (head) dimension
   float* partial;            // [batch][tiles_m][tiles_n][splits][BN][BM] when splits > 1
   int tiles_m, tiles_n, batch;
+  // The weights (A) were not written by the kernel before this one, nor by
+  // anything still running: the first STAGES stages' weight tiles are
+  // requested before the programmatic wait.
+  int pre_a;
 };
 
 template <int BN>
@@ -108,8 +112,29 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  pdl_trigger();
+  // The weight halves of the first stages go out while the previous kernel
+  // finishes (every kernel here lets its successor launch only once it has
+  // passed its own wait, so nothing older than the previous kernel is still
+  // running, and that one does not write weights); the activation halves
+  // follow the wait, completing the same barriers.
+  uint32_t pre = 0;
+  if (g.pre_a && warp == 0) {
+    for (int item = blockIdx.x; item < items && pre < (uint32_t)STAGES; item += gridDim.x) {
+      int bz, split, tm, tn;
+      decode(item, bz, split, tm, tn);
+      const int nk = ksteps(split);
+      for (int kt = 0; kt < nk && pre < (uint32_t)STAGES; ++kt, ++pre) {
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full[pre], STAGE);
+          tma_load_2d(smem + pre * STAGE, &mapA, split * g.kchunk + kt * BK, bz * g.a_batch_rows + tm * BM,
+                      &full[pre]);
+        }
+        __syncwarp();
+      }
+    }
+  }
   pdl_wait();  // the activations (and the split-K scratch) come from the previous kernel
+  pdl_trigger();
 
   if (warp == 0) {
     // TMA producer: runs ahead across items as far as the ring allows.
@@ -121,11 +146,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int nk = ksteps(split);
       for (int kt = 0; kt < nk; ++kt, ++cnt) {
         const int s = cnt % STAGES;
-        if (!(ok = mbar_wait_warp(&empty[s], ((cnt / STAGES) & 1) ^ 1, abort_flag, nullptr))) break;
+        const bool a_done = cnt < pre;  // weight half already requested before the wait
+        if (!a_done && !(ok = mbar_wait_warp(&empty[s], ((cnt / STAGES) & 1) ^ 1, abort_flag, nullptr))) break;
         if (elect_one()) {
-          mbar_arrive_expect_tx(&full[s], STAGE);
           const int k = split * g.kchunk + kt * BK;
-          tma_load_2d(smem + s * STAGE, &mapA, k, bz * g.a_batch_rows + tm * BM, &full[s]);
+          if (!a_done) {
+            mbar_arrive_expect_tx(&full[s], STAGE);
+            tma_load_2d(smem + s * STAGE, &mapA, k, bz * g.a_batch_rows + tm * BM, &full[s]);
+          }
           if (g.b_is_3d) tma_load_3d(smem + s * STAGE + A_BYTES, &mapB, k, bz, tn * BN, &full[s]);
           else tma_load_2d(smem + s * STAGE + A_BYTES, &mapB, k, tn * BN, &full[s]);
         }
@@ -248,8 +276,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 constexpr int MAX_SPLITS = 32;
 template <int BN, class Epi>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const Args g, const Epi epi) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int bz = blockIdx.z, slices = BN / 8;
   const int tile_m = blockIdx.x >> 1, half = blockIdx.x & 1;
   const int tile_n = blockIdx.y / slices, slice = blockIdx.y % slices;

@@ -333,7 +333,7 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, long long dim0, long lon
 template <int BN, class Epi>
 cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                            int M, int N, int K, int batch, const Epi& epi, float* partial, long long partial_floats,
-                           cudaStream_t st, int max_ctas) {
+                           cudaStream_t st, int max_ctas, bool pre_a) {
   CUtensorMap mapW, mapX;
   // Weights: batches are contiguous row blocks of N rows.
   if (batch > 1 && sB != (long long)N * ldb) return cudaErrorInvalidValue;
@@ -355,7 +355,7 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
   const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
   splits = ceil_div(K, kchunk);
-  gemm_tc::Args g{N, M, K, splits, kchunk, N, x3d ? 1 : 0, partial, tm, tn, batch};
+  gemm_tc::Args g{N, M, K, splits, kchunk, N, x3d ? 1 : 0, partial, tm, tn, batch, pre_a ? 1 : 0};
   const size_t smem = gemm_tc::smem_bytes<BN>();
   auto kfn = gemm_tc::gemm_tc_kernel<BN, Epi>;
   cudaError_t e = set_smem_once(kfn, smem);
@@ -379,19 +379,22 @@ cudaError_t gemm_simt(const void* A, long long lda, long long sA, const void* B,
                       int tile_split_cap);
 
 // `max_ctas` caps the CTAs of the tensor-core GEMM (a GEMM sharing the GPU
-// with another stream's).
+// with another stream's).  `pre_a`: the kernel before this one in the stream
+// is one of this call's own (which writes no weights), so the GEMM may
+// request its first weight tiles before its programmatic wait.
 template <typename T, class Epi>
 cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long long ldb, long long sB,
                  int M, int N, int K, int batch, const Epi& epi, void* ws, const Plan& P,
-                 cudaStream_t st, int tile_split_cap = kSplitKTileSplits, int max_ctas = INT_MAX) {
+                 cudaStream_t st, int tile_split_cap = kSplitKTileSplits, int max_ctas = INT_MAX,
+                 bool pre_a = false) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if constexpr (sizeof(T) == 2) {
     const long long cap = (long long)tile_split_cap * 64 * 64;
     if (M <= 512)
       return gemm_tc_launch<64>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
-                                max_ctas);
+                                max_ctas, pre_a);
     return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
-                               max_ctas);
+                               max_ctas, pre_a);
   } else {
     return gemm_simt(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, ws, P, st, tile_split_cap);
   }
@@ -575,14 +578,15 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
     epi.n_h = d.n_h; epi.d_h = d.d_h; epi.d_r = d.d_r; epi.d_c = d.d_c; epi.d_cr = q_row;
     epi.qabs_rows = P.qrows; epi.n_q = n_q; epi.prefill_S = prefill_S;
     epi.qr_scale = qscale;
-    if ((e = gemm<T>(src, din, 0, w->uqr, din, 0, R, d.n_h * (d.d_h + d.d_r), din, 1, epi, ws, P, st)))
+    if ((e = gemm<T>(src, din, 0, w->uqr, din, 0, R, d.n_h * (d.d_h + d.d_r), din, 1, epi, ws, P, st,
+                     kSplitKTileSplits, INT_MAX, d.d_cq > 0)))
       return cuda_status(e);
   }
   // (3) absorption q~_h = W_UK,h^T q_C,h, scaled.
   {
     EpiStore<T> epi{at<T>(ws, P.qabs), (long long)P.qrows * q_row, q_row, qscale};
     if ((e = gemm<T>(at<T>(ws, P.qc), (long long)d.n_h * d.d_h, d.d_h, w->ukt, d.d_h, (long long)d.d_c * d.d_h,
-                     R, d.d_c, d.d_h, d.n_h, epi, ws, P, st)))
+                     R, d.d_c, d.d_h, d.n_h, epi, ws, P, st, kSplitKTileSplits, INT_MAX, true)))
       return cuda_status(e);
   }
   // The schedule has run on the side stream beside steps (1) - (3).
@@ -632,7 +636,7 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   {
     EpiStore<float> epi{out, (long long)d.n_h * d.d_v, d.d_v, 1.f};
     if ((e = gemm<T>(at<T>(ws, P.obar), (long long)d.n_h * d.d_c, d.d_c, w->uv, d.d_c, (long long)d.d_v * d.d_c,
-                     R, d.d_v, d.d_c, d.n_h, epi, ws, P, st)))
+                     R, d.d_v, d.d_c, d.n_h, epi, ws, P, st, kSplitKTileSplits, INT_MAX, true)))
       return cuda_status(e);
   }
   return MLA_OK;

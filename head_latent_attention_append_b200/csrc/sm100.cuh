@@ -107,10 +107,13 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel of its stream is finishing.  pdl_wait() blocks until
 // that kernel has completed and its memory operations are visible: every
-// kernel calls it before its first global-memory access, so only prologue
-// work (barrier init, TMEM allocation, descriptor prefetch) overlaps.  In a
-// kernel launched without the attribute it returns at once.
-// pdl_trigger() lets the next kernel in the stream begin launching.
+// kernel calls it before its first global-memory access (the one exception:
+// a projection GEMM's weight loads, which its caller marks safe), so only
+// prologue work (barrier init, TMEM allocation, descriptor prefetch) and
+// those weight loads overlap.  In a kernel launched without the attribute it
+// returns at once.  pdl_trigger() lets the next kernel in the stream begin
+// launching; every kernel calls it only after its own pdl_wait(), so when a
+// kernel starts, everything before its predecessor has completed.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
