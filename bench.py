@@ -240,6 +240,52 @@ def measured_traffic(workload: str):
     return rec["traffic_bytes"] if kernel_code_hash(rec["source_files"]) == rec["source_sha256"] else None
 
 
+def e2e_pipelined(s, step_on, h_host, args, ws, stream) -> float:
+    """ms per step of the public-API loop with each step's host->device copy
+    of its inputs and device->host copy of its outputs on two copy streams,
+    double-buffered, so that they overlap the neighbouring steps' compute.
+    The timed region runs from the first copy in to the last copy out."""
+    import torch
+    cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+    h_dev = [s.h_new, s.h_new.clone()]
+    out_dev = [s.out, torch.empty_like(s.out)]
+    out_host = [torch.empty(s.out.shape, dtype=s.out.dtype).pin_memory() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            j = i & 1
+            if i >= 2:
+                cs_in.wait_event(ev_c[j])      # step i-2 no longer reads h_dev[j]
+            with torch.cuda.stream(cs_in):
+                h_dev[j].copy_(h_host, non_blocking=True)
+            ev_in[j].record(cs_in)
+            stream.wait_event(ev_in[j])
+            if i >= 2:
+                stream.wait_event(ev_out[j])   # step i-2's outputs have left out_dev[j]
+            s.h_new, s.out = h_dev[j], out_dev[j]
+            step_on(i)
+            ev_c[j].record(stream)
+            cs_out.wait_event(ev_c[j])
+            with torch.cuda.stream(cs_out):
+                out_host[j].copy_(out_dev[j], non_blocking=True)
+            ev_out[j].record(cs_out)
+
+    run(args.warmup)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cs_in)
+    run(args.steps)
+    e1.record(cs_out)
+    torch.cuda.synchronize()
+    s.h_new, s.out = h_dev[0], out_dev[0]
+    return max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
+
+
 PREFILL_SAMPLE_TOKENS = 1024   # causal prefix of one sequence per oracle prefill sample
 
 
@@ -525,6 +571,13 @@ def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
     ms_e2e_graph = max_over_ranks(e2.elapsed_time(e3) / args.steps, ws)
     del graphs, g2s
 
+    # The same end-to-end steps as a serving loop runs them: step i's inputs
+    # go up on a copy stream while step i-1 computes, and its outputs come
+    # down on another while step i+1 computes (two device and two pinned
+    # host buffers; every step's copies are still inside the timed region,
+    # which runs from the first copy in to the last copy out).
+    ms_e2e_pipe = e2e_pipelined(s, step_on, h_host, args, ws, stream)
+
     tokens = wl.B * wl.n_q
     attn_avg_ms = attn_ms / max(1, attn_n)
     hbm_gbs = unique_bytes / (attn_avg_ms * 1e-3) / 1e9
@@ -566,10 +619,14 @@ def measure_workload(name, args, ws, local, peaks, with_cpu_baseline):
         "attention_tflops": ws * flops / (ms_step * 1e-3) / 1e12,
         "form": "materialised" if wl.materialised else "absorbed",
         "roofline": roofline,
-        "e2e": {"value": ws * units / (ms_e2e * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-                "timing": "eager C-ABI calls every step, copies included",
-                "graph": {"value": ws * units / (ms_e2e_graph * 1e-3) / scale, "ms_per_step": ms_e2e_graph}},
+        "e2e": {"value": ws * units / (ms_e2e_pipe * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e_pipe,
+                "timing": ("eager C-ABI calls every step, each step's copy in and copy out included, on copy "
+                           "streams overlapping the neighbouring steps' compute (double-buffered)"),
+                "serial": {"value": ws * units / (ms_e2e * 1e-3) / scale, "ms_per_step": ms_e2e,
+                           "timing": "copy in, step, copy out one after another on one stream"},
+                "graph": {"value": ws * units / (ms_e2e_graph * 1e-3) / scale, "ms_per_step": ms_e2e_graph,
+                          "timing": "the serial form as a replayed graph"}},
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }
