@@ -63,7 +63,7 @@ extern "C" {
 typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = -1,    /* null pointer, bad size, misaligned buffer   */
-  MLA_ERR_UNSUPPORTED = -2,    /* dimensions this build has no kernel for     */
+  MLA_ERR_UNSUPPORTED = -2,    /* dimensions the library has no kernel for    */
   MLA_ERR_WORKSPACE = -3,      /* workspace or weight buffer too small        */
   MLA_ERR_CUDA = -4,           /* a CUDA runtime call failed                  */
   MLA_ERR_DEVICE_BOUNDS = -5,  /* device-side check: index out of range       */
@@ -82,7 +82,7 @@ typedef struct {
   int d_cq;             /* query latent width; 0 = no query latent           */
   float rope_base;      /* e.g. 10000                                        */
   float softmax_scale;  /* 0 selects 1/sqrt(d_h + d_r) on both score terms   */
-  int page_size;        /* tokens per cache page; this build supports 64     */
+  int page_size;        /* tokens per cache page; the library supports 64    */
   mla_dtype dtype;      /* element type of weights, hidden states and cache  */
   int rope_key_per_head; /* 0: one RoPE key shared by all heads (default);
                             1: one d_r key per head (see below)              */
