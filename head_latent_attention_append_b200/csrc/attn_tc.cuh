@@ -62,6 +62,14 @@
 // its row max through shared memory and a 128-thread named barrier, and each
 // keeps a partial row sum (the same rescalings), added at the end.  Every
 // wait is bounded (sm100::mbar_wait).
+//
+// A worker walks its schedule segments (sched.cuh).  At a segment's end the
+// softmax warps load the next segment's Q rows, then write this segment's O:
+// normalised into obar for a whole row block, or for a piece of a split row
+// block into its partial slot with its (m, l).  When the launch passes
+// arrival counters (AttnArgs::arrive), each piece then counts in, and the
+// last piece of a row block to do so merges every piece's slot into obar
+// (otherwise combine_kernel does it after the launch).
 #pragma once
 #include "attn_simt.cuh"
 #include "sm100.cuh"
