@@ -56,6 +56,24 @@ __host__ __device__ __forceinline__ long long ml_index(int slot, int half, int n
 namespace attn_simt {
 constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
 
+// The eight bf16 (or four fp32) values of a 16-byte load, as floats.
+template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+    f[2 * q] = v.x;
+    f[2 * q + 1] = v.y;
+  }
+}
+template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, float* f) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) {
   extern __shared__ float smem[];
@@ -72,6 +90,7 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
   const T* qabs = static_cast<const T*>(a.qabs);
   const T* cache = static_cast<const T*>(a.cache);
   const Sched& S = a.sched;
+  const bool vec_rows = ((a.d_cr * (int)sizeof(T)) & 15) == 0 && (reinterpret_cast<uintptr_t>(cache) & 15) == 0;
 
   for (int si = S.worker_seg[w]; si < S.worker_seg[w + 1]; ++si) {
     const Seg g = S.segs[si];
@@ -94,18 +113,51 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
     const int k_end = min(nkeys, g.t_hi * a.page_size);
     for (int k0 = k_begin; k0 < k_end; k0 += KC) {
       __syncthreads();
-      // Stage KC cache rows (positions k0 .. k0+KC-1) through the page table.
-      for (int i = tid; i < KC * a.d_cr; i += THREADS) {
-        int k = i / a.d_cr, j = i % a.d_cr, p = k0 + k;
-        float v = 0.f;
-        if (p < k_end) {
-          int page = a.page_table[(long long)seq * a.max_pages + p / a.page_size];
-          if (page >= 0 && page < a.num_pages)
-            v = to_f32(cache[((long long)page * a.page_size + p % a.page_size) * a.d_cr + j]);
-          else if (j == 0)
-            flag_error(a.err, kErrBounds);
+      // Stage KC cache rows (positions k0 .. k0+KC-1) through the page table:
+      // each warp takes RPW rows, looks up their pages first (one load per
+      // row for the whole warp), then reads the rows with 16-byte loads when
+      // every row starts on a 16-byte boundary, element by element if not.
+      {
+        constexpr int RPW = KC / (THREADS / 32);
+        constexpr int EPV = 16 / (int)sizeof(T);  // elements per 16-byte load
+        const T* src[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const int p = k0 + warp * RPW + r;
+          src[r] = nullptr;
+          if (p < k_end) {
+            const int page = a.page_table[(long long)seq * a.max_pages + p / a.page_size];
+            if (page >= 0 && page < a.num_pages)
+              src[r] = cache + ((long long)page * a.page_size + p % a.page_size) * a.d_cr;
+            else if (lane == 0)
+              flag_error(a.err, kErrBounds);
+          }
         }
-        Cs[k * pitch + j] = v;
+        if (vec_rows) {
+          const int nv = a.d_cr / EPV;
+          for (int v0 = 0; v0 < nv; v0 += 32) {
+            const int v = v0 + lane;
+            uint4 u[RPW];
+#pragma unroll
+            for (int r = 0; r < RPW; ++r)
+              u[r] = (src[r] && v < nv) ? __ldg(reinterpret_cast<const uint4*>(src[r]) + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+              if (v >= nv) continue;
+              float f[EPV];
+              unpack16<T>(u[r], f);
+              float* crow = Cs + (warp * RPW + r) * pitch + v * EPV;
+#pragma unroll
+              for (int e = 0; e < EPV; ++e) crow[e] = f[e];
+            }
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < RPW; ++r) {
+            float* crow = Cs + (warp * RPW + r) * pitch;
+            for (int j = lane; j < a.d_cr; j += 32) crow[j] = src[r] ? to_f32(src[r][j]) : 0.f;
+          }
+        }
       }
       __syncthreads();
       // Scores for HG x KC (head, key) pairs.
