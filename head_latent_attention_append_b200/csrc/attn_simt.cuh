@@ -56,6 +56,11 @@ __host__ __device__ __forceinline__ long long ml_index(int slot, int half, int n
 namespace attn_simt {
 constexpr int THREADS = 256, KC = 32, MAX_CPT = 32;
 
+// Staged rows (cache rows and Q rows, fp32) are padded to 4 mod 32 floats:
+// 16-byte aligned, and the 32 rows of a warp's score loads start in eight
+// different 4-bank groups (conflict-free 16-byte loads).
+__host__ __device__ constexpr int row_pitch(int d_cr) { return (d_cr + 31) / 32 * 32 + 4; }
+
 // The eight bf16 (or four fp32) values of a 16-byte load, as floats.
 template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float* f);
 template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
@@ -77,7 +82,7 @@ template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, floa
 template <typename T>
 __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) {
   extern __shared__ float smem[];
-  const int pitch = a.d_cr + 1;        // cache rows; a Q row uses the first q_row of its pitch
+  const int pitch = row_pitch(a.d_cr);  // cache rows; a Q row uses the first q_row of its pitch
   float* Qs = smem;                    // [HG][pitch]
   float* Cs = Qs + HG * pitch;         // [KC][pitch]
   float* Ps = Cs + KC * pitch;         // [HG][KC]
@@ -87,6 +92,10 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
   const int TPH = THREADS / HG;        // threads per head in the output update
   const int oh = tid / TPH, oj = tid % TPH;
   const int cpt = ceil_div(a.d_c, TPH);  // <= MAX_CPT (d_c <= 512, TPH >= 16)
+  // d_c % 4 == 0: the latent columns are read four at a time (16-byte
+  // shared-memory loads), and an output thread owns groups of four columns.
+  const bool vec_c = (a.d_c & 3) == 0;
+  const int cpt4 = ceil_div(a.d_c / 4, TPH);  // <= MAX_CPT / 4
   const T* qabs = static_cast<const T*>(a.qabs);
   const T* cache = static_cast<const T*>(a.cache);
   const Sched& S = a.sched;
@@ -167,7 +176,20 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
         const float* c = Cs + k * pitch;
         const float* kr = c + a.d_c + (a.rope_per_head ? (h0 + h) * a.d_r : 0);
         float acc = 0.f;
-        for (int j = 0; j < a.d_c; ++j) acc = fmaf(q[j], c[j], acc);
+        if (vec_c) {
+          float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j = 0; j < a.d_c; j += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(q + j);
+            const float4 cv = *reinterpret_cast<const float4*>(c + j);
+            s4.x = fmaf(qv.x, cv.x, s4.x);
+            s4.y = fmaf(qv.y, cv.y, s4.y);
+            s4.z = fmaf(qv.z, cv.z, s4.z);
+            s4.w = fmaf(qv.w, cv.w, s4.w);
+          }
+          acc = (s4.x + s4.y) + (s4.z + s4.w);
+        } else {
+          for (int j = 0; j < a.d_c; ++j) acc = fmaf(q[j], c[j], acc);
+        }
         for (int j = 0; j < a.d_r; ++j) acc = fmaf(q[a.d_c + j], kr[j], acc);
         Ps[h * KC + k] = (k0 + k < k_end) ? acc : -INFINITY;
       }
@@ -198,14 +220,37 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
       if (oh < HG) {
         const float corr = st[oh * 3 + 2];
         const float* P = Ps + oh * KC;
+        if (vec_c) {
 #pragma unroll
-        for (int r = 0; r < MAX_CPT; ++r) {
-          if (r < cpt && oj + r * TPH < a.d_c) {
-            int j = oj + r * TPH;
-            float acc = o[r] * corr;
+          for (int r = 0; r < MAX_CPT / 4; ++r) {
+            const int g4 = oj + r * TPH;
+            if (r < cpt4 && 4 * g4 < a.d_c) {
+              float4 acc = make_float4(o[4 * r] * corr, o[4 * r + 1] * corr, o[4 * r + 2] * corr, o[4 * r + 3] * corr);
 #pragma unroll 8
-            for (int k = 0; k < KC; ++k) acc = fmaf(P[k], Cs[k * pitch + j], acc);
-            o[r] = acc;
+              for (int k = 0; k < KC; ++k) {
+                const float pk = P[k];
+                const float4 cv = *reinterpret_cast<const float4*>(Cs + k * pitch + 4 * g4);
+                acc.x = fmaf(pk, cv.x, acc.x);
+                acc.y = fmaf(pk, cv.y, acc.y);
+                acc.z = fmaf(pk, cv.z, acc.z);
+                acc.w = fmaf(pk, cv.w, acc.w);
+              }
+              o[4 * r] = acc.x;
+              o[4 * r + 1] = acc.y;
+              o[4 * r + 2] = acc.z;
+              o[4 * r + 3] = acc.w;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < MAX_CPT; ++r) {
+            if (r < cpt && oj + r * TPH < a.d_c) {
+              int j = oj + r * TPH;
+              float acc = o[r] * corr;
+#pragma unroll 8
+              for (int k = 0; k < KC; ++k) acc = fmaf(P[k], Cs[k * pitch + j], acc);
+              o[r] = acc;
+            }
           }
         }
       }
@@ -216,18 +261,18 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
     if (oh < HG && h0 + oh < a.n_h) {
       const int h = h0 + oh;
       const float m = st[oh * 3 + 0], l = st[oh * 3 + 1];
-      if (g.slot < 0) {
-        T* out = static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c;
-        const float inv = 1.f / l;
+      // Column of o[r]: groups of four (4 (oj + (r / 4) TPH) + r % 4) when
+      // vec_c, else oj + r TPH.
+      T* dst = g.slot < 0 ? static_cast<T*>(a.obar) + ((long long)rb * a.n_h + h) * a.d_c
+                          : static_cast<T*>(a.part_o) + ((long long)g.slot * a.n_h + h) * a.d_c;
+      const float inv = 1.f / l;
 #pragma unroll
-        for (int r = 0; r < MAX_CPT; ++r)
-          if (r < cpt && oj + r * TPH < a.d_c) out[oj + r * TPH] = from_f32<T>(o[r] * inv);
-      } else {
-        T* po = static_cast<T*>(a.part_o) + ((long long)g.slot * a.n_h + h) * a.d_c;
-        const float inv = 1.f / l;
-#pragma unroll
-        for (int r = 0; r < MAX_CPT; ++r)
-          if (r < cpt && oj + r * TPH < a.d_c) po[oj + r * TPH] = from_f32<T>(o[r] * inv);
+      for (int r = 0; r < MAX_CPT; ++r) {
+        const int col = vec_c ? 4 * (oj + (r / 4) * TPH) + (r % 4) : oj + r * TPH;
+        const bool mine = vec_c ? (r / 4 < cpt4 && col < a.d_c) : (r < cpt && col < a.d_c);
+        if (mine) dst[col] = from_f32<T>(o[r] * inv);
+      }
+      if (g.slot >= 0) {
         if (oj == 0) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -241,7 +286,7 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(AttnArgs a, int HG) 
 }
 
 inline size_t smem_bytes(int HG, int d_cr) {
-  return sizeof(float) * ((size_t)(HG + KC) * (d_cr + 1) + HG * KC + HG * 3);
+  return sizeof(float) * ((size_t)(HG + KC) * row_pitch(d_cr) + HG * KC + HG * 3);
 }
 }  // namespace attn_simt
 
