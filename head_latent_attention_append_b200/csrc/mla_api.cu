@@ -523,8 +523,10 @@ mla_status attend_impl(const mla_weights* w, const void* hq, const int32_t* kv_l
   while (HG > d.n_h) HG >>= 1;
   const int G = kTensorCores ? 2 : ceil_div(d.n_h, HG);
   // bf16: one CTA pair per two SMs (one CTA per SM; all of TMEM each).
+  // CUDA-core kernel: one CTA per SM and head group (its registers and the
+  // staged rows fill an SM), so every worker runs in a single round.
   int W = kTensorCores ? std::max(1, std::min(kWorkerSlots, num_sms() / 2))
-                       : std::max(1, std::min(kWorkerSlots, (2 * num_sms()) / G));
+                       : std::max(1, std::min(kWorkerSlots, num_sms() / G));
   // bf16 without context parallelism, with at least half as many row blocks
   // as workers (so a split row block has two or three pieces): the attention
   // kernel merges split row blocks itself (a row block has at most one piece
