@@ -346,12 +346,13 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   }
   const int tm = ceil_div(N, gemm_tc::BM), tn = ceil_div(M, BN), tiles = tm * tn * batch;
   const int nk = ceil_div(K, gemm_tc::BK);
-  // Few output tiles (decode): split K so that about two work items per SM
-  // keep every SM streaming weights; the reduce kernel sums the splits in
-  // order and runs the epilogue.
+  // Few output tiles (decode): split K so that every SM streams weights in a
+  // single round (one work item per SM; two per SM measured 1-2 us slower
+  // on the decode step); the reduce kernel sums the splits in order and runs
+  // the epilogue.
   int splits = 1;
   const int sms = std::min(num_sms(), max_ctas);
-  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), ceil_div(2 * sms, tiles));
+  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), std::max(1, sms / tiles));
   while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
   const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
   splits = ceil_div(K, kchunk);
