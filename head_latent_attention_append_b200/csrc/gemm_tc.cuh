@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ends up with 8 consecutive weight rows (output columns) of one token:
     // the functor then writes them as one 16-byte (bf16) or 32-byte (fp32)
     // vector.
-    const int q = warp & 3, lane = tid & 31, r = q * 32 + lane;
+    const int q = warp & 3, lane = tid & 31;
     const int part = (warp - 2) / 4, c_lo = part * (BN / 4), c_hi = c_lo + BN / 4;
     float* stg = epi_stage + (warp - 2) * (8 * EPI_PITCH);
     const int tj = lane >> 2, rg = (lane & 3) * 8;  // token and first row this lane stores

@@ -9,6 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cstring>
 #include <mutex>
 #include <utility>
 
@@ -284,46 +285,83 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Every map here is a bf16 tensor of rank 2 or 3, 128-byte swizzle, no
+// interleave, 256-byte L2 promotion, zero fill; it is a pure function of
+// (base, dims, byte strides, box).  The last kMapCache encodings of this host
+// thread are kept, so a steady stream of calls on the same buffers does not
+// re-encode its dozen maps every step.
+constexpr int kMapCache = 32;
+struct MapKey {
+  const void* base;
+  int rank;
+  cuuint64_t dim[3], stride[2];
+  cuuint32_t box[3];
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rank == o.rank && std::memcmp(dim, o.dim, sizeof dim) == 0 &&
+           std::memcmp(stride, o.stride, sizeof stride) == 0 && std::memcmp(box, o.box, sizeof box) == 0;
+  }
+};
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  int used = 0, next = 0;
+};
+thread_local MapCache g_maps;
+
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dim, const cuuint64_t* stride,
+                 const cuuint32_t* box) {
+  MapKey k{};
+  k.base = base;
+  k.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    k.dim[i] = dim[i];
+    k.box[i] = box[i];
+    if (i + 1 < rank) k.stride[i] = stride[i];
+  }
+  for (int i = 0; i < g_maps.used; ++i)
+    if (g_maps.key[i] == k) {
+      *map = g_maps.map[i];
+      return true;
+    }
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  if (fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), k.dim, k.stride, k.box,
+         es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = g_maps.next;
+  g_maps.key[slot] = k;
+  g_maps.map[slot] = *map;
+  g_maps.next = (slot + 1) % kMapCache;
+  if (g_maps.used < kMapCache) ++g_maps.used;
+  return true;
+}
+
 // The cache as a 2-D tensor [rows = num_pages * 64][d_cr] bf16, read in boxes
 // of 64 columns x `box_rows` rows with 128-byte swizzle.  Columns past d_cr
 // read as zero (the RoPE chunk of a row narrower than 64 columns).
 bool encode_cache_map(CUtensorMap* map, const void* cache, int d_cr, long long rows, int box_rows) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)d_cr, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)d_cr * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(cache), gdim, gstride, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_bf16(map, cache, 2, gdim, gstride, box);
 }
 
 // bf16 tensor maps with 128-byte swizzle for the projection GEMMs.
 bool encode_bf16_2d(CUtensorMap* map, const void* base, long long dim0, long long dim1, long long stride1_elems,
                     int box0, int box1) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)dim0, (cuuint64_t)dim1};
   cuuint64_t gstride[1] = {(cuuint64_t)stride1_elems * 2};
   cuuint32_t box[2] = {(cuuint32_t)box0, (cuuint32_t)box1};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_bf16(map, base, 2, gdim, gstride, box);
 }
 bool encode_bf16_3d(CUtensorMap* map, const void* base, long long dim0, long long dim1, long long dim2,
                     long long stride1_elems, long long stride2_elems, int box0, int box1, int box2) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
   cuuint64_t gdim[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
   cuuint64_t gstride[2] = {(cuuint64_t)stride1_elems * 2, (cuuint64_t)stride2_elems * 2};
   cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, (cuuint32_t)box2};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_bf16(map, base, 3, gdim, gstride, box);
 }
 
 // tcgen05 projection GEMM: C[b][m][n] = sum_k A[b][m][k] * B[b][n][k] with A
