@@ -38,7 +38,7 @@ struct Args {
 
 template <int BN>
 __host__ __device__ constexpr int stages() {
-  return BN == 64 ? 8 : 6;
+  return BN == 64 ? 8 : (BN == 128 ? 6 : 4);
 }
 // Per epilogue warp: 8 tokens x 32 rows of fp32, each token's row padded to
 // 36 floats so that the transposed reads fall in different bank groups.

@@ -432,7 +432,12 @@ cudaError_t gemm(const void* A, long long lda, long long sA, const void* B, long
     if (M <= 512)
       return gemm_tc_launch<64>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
                                 max_ctas, pre_a);
-    return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
+    if (M < 4096)
+      return gemm_tc_launch<128>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
+                                 max_ctas, pre_a);
+    // Many tokens (prefill): 256-token tiles, so each 48 KB stage (weights
+    // 16 KB, tokens 32 KB) feeds twice the tensor work of a 128-token one.
+    return gemm_tc_launch<256>(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, at<float>(ws, P.partial), cap, st,
                                max_ctas, pre_a);
   } else {
     return gemm_simt(A, lda, sA, B, ldb, sB, M, N, K, batch, epi, ws, P, st, tile_split_cap);
