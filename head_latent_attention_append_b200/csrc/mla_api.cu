@@ -61,7 +61,7 @@ void prof_mark(cudaStream_t st, bool start) {
 constexpr int kWorkerSlots = 296;        // partial-slot capacity: 2 * kWorkerSlots
 constexpr int kSplitKTileSplits = 1024;  // split-K scratch: tiles * splits <= this
 constexpr int kCounterCap = 1024;
-constexpr int kSideTileSplits = 256;     // split-K scratch of the side-stream append (tiles * splits)
+constexpr int kSideTileSplits = 1024;    // split-K scratch of the side-stream append (tiles * splits): as the main one's
 constexpr int kSideAppendCtas = 32;      // CTAs of the side-stream append GEMM
 constexpr double kLog2e = 1.4426950408889634074;
 
@@ -389,8 +389,12 @@ cudaError_t gemm_tc_launch(const void* A, long long lda, long long sA, const voi
   // on the decode step); the reduce kernel sums the splits in order and runs
   // the epilogue.
   int splits = 1;
+  // The split count depends on the GPU, not on `max_ctas`, so a GEMM capped
+  // to a few CTAs (the side-stream append) sums its partials exactly as the
+  // uncapped one does: the same cache rows, bit for bit.
   const int sms = std::min(num_sms(), max_ctas);
-  if (2 * tiles < sms) splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), std::max(1, sms / tiles));
+  if (2 * tiles < num_sms())
+    splits = std::min(std::min(gemm_tc::MAX_SPLITS, nk), std::max(1, num_sms() / tiles));
   while (splits > 1 && (long long)tiles * splits * BN * gemm_tc::BM > partial_floats) --splits;
   const int kchunk = ceil_div(nk, splits) * gemm_tc::BK;
   splits = ceil_div(K, kchunk);
